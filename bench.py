@@ -1,0 +1,457 @@
+"""Benchmark of the Sparse VideoGen attention step on B200.
+
+Default workload: HunyuanVideo 720p 5 s shape (B=1, H=24, d=128, 33 latent
+frames of 45x80 = 118,800 video tokens + 256 text tokens), one full step per
+iteration: QK-Norm + 3D RoPE -> online profiling -> block index -> layout
+transform -> block-sparse attention -> inverse layout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--sweep]
+
+Prints one JSON line (rank 0).  `value` is effective TFLOP/s: the FLOPs of
+QK^T and PV over the kept 128x64 tiles (4*d*rows*cols per tile) divided by the
+whole step's device time.  With N > 1 (torchrun) every rank runs its own
+independent layer (weak scaling, no data-path collective); time is the max
+over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import svg_workloads as W  # noqa: E402
+
+METRIC = "sparse-attn layer ms and effective TFLOP/s (% bf16 peak) at 118,800 tokens"
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 7700.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: d[k] for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def kept_tile_flops(row_ptr: np.ndarray, col: np.ndarray, wl) -> float:
+    """4*d*rows*cols summed over the listed (q-block, k-block) tiles."""
+    nqb = wl.nqb
+    counts = np.diff(row_ptr.astype(np.int64))
+    qb = np.tile(np.arange(nqb), wl.B * wl.H)
+    rows = np.minimum(wl.bq, wl.L - qb * wl.bq)
+    cols = np.minimum(wl.bk, wl.L - col.astype(np.int64) * wl.bk)
+    # every listed tile of one q-block has `rows` query rows
+    per_entry_rows = np.repeat(rows, counts)
+    return float(4.0 * wl.d * np.sum(per_entry_rows * cols))
+
+
+def traffic_from_profile(kernel_file: str, summary: str):
+    """DRAM bytes per launch recorded in a committed ncu summary, if it was
+    taken on the current kernel source (sha256 match); else None."""
+    p = os.path.join(ROOT, "profiles", summary)
+    src = os.path.join(ROOT, "sparse_attention_video_qk_b200", "csrc", kernel_file)
+    if not (os.path.exists(p) and os.path.exists(src)):
+        return None
+    text = open(p).read()
+    m_sha = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    m_b = re.search(r"traffic_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
+    if not (m_sha and m_b):
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != m_sha.group(1):
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU arm --
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_attention_video_qk_b200 as svg
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    wl = W.CONFIGS[args.config]
+    pb = svg.Problem.from_workload(wl)
+    inp = W.make_inputs(wl, seed=wl.seed + rank)          # each rank: its own layer
+    pin = lambda a, bf=True: (torch.from_numpy(a).view(torch.bfloat16) if bf else torch.from_numpy(a)).pin_memory()
+    q_h, k_h, v_h = pin(inp["q"]), pin(inp["k"]), pin(inp["v"])
+    gq_h, gk_h, si_h = pin(inp["gamma_q"], False), pin(inp["gamma_k"], False), pin(inp["sample_idx"], False)
+    del inp
+    q, k, v = (t.to(device) for t in (q_h, k_h, v_h))
+    gq, gk, si = gq_h.to(device), gk_h.to(device), si_h.to(device)
+    buf = svg.StepBuffers(pb, int(si.numel()), device)
+    stream = torch.cuda.current_stream()
+    lib = svg.lib()
+    sh, pr = pb.c_shape(), pb.c_params()
+    cs = ctypes.c_void_p(stream.cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+    def stage_calls():
+        """The step as its six C-ABI calls (same as svg_attention_step)."""
+        b = buf
+        return [
+            ("qknorm_rope", lambda: lib.svg_qknorm_rope_layout(ctypes.byref(sh), ctypes.byref(pr), 1, P(q), P(k), None,
+                                                              P(gq), P(gk), P(b.table), None, P(b.qn), P(b.kn), None,
+                                                              cs)),
+            ("profile", lambda: lib.svg_profile_heads(ctypes.byref(sh), ctypes.byref(pr), P(b.qn), P(b.kn), P(v),
+                                                      P(si), int(si.numel()), P(b.workspace), b.workspace.numel(),
+                                                      P(b.mse), P(b.kinds), cs)),
+            ("block_index", lambda: lib.svg_build_block_index(ctypes.byref(sh), ctypes.byref(pr), P(b.kinds),
+                                                              P(b.row_ptr), P(b.col), P(b.full), b.capacity, cs)),
+            ("layout", lambda: lib.svg_qknorm_rope_layout(ctypes.byref(sh), ctypes.byref(pr), 2, P(b.qn), P(b.kn),
+                                                          P(v), None, None, None, P(b.kinds), P(b.qp), P(b.kp),
+                                                          P(b.vp), cs)),
+            ("attention", lambda: lib.svg_block_sparse_attn(ctypes.byref(sh), ctypes.byref(pr), P(b.qp), P(b.kp),
+                                                            P(b.vp), P(b.kinds), P(b.row_ptr), P(b.col), P(b.full),
+                                                            P(b.op), None, cs)),
+            ("inverse_layout", lambda: lib.svg_inverse_layout(ctypes.byref(sh), P(b.kinds), P(b.op), P(b.out), cs)),
+        ]
+
+    calls = stage_calls()
+    launches_per_step = 1 + 2 + 3 + 1 + 1 + 1
+
+    def one_step(events=None):
+        for i, (name, fn) in enumerate(calls):
+            st = fn()
+            if st != 0:
+                raise svg.SVGError(st, name)
+            if events is not None:
+                events[i + 1].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    svg.sync_status()
+    flops = kept_tile_flops(buf.row_ptr.cpu().numpy(), buf.col[: int(buf.row_ptr[-1])].cpu().numpy(), wl)
+    kinds = buf.kinds.cpu().numpy()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        t_start.record(stream)
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            one_step(ev[s])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    svg.sync_status()
+    total_ms = t_start.elapsed_time(t_end)
+    stage_ms = {name: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps))
+                for i, (name, _) in enumerate(calls)}
+    clocks = clk.summary()
+
+    # ---- end to end through the public host-buffer API (copies inside the timed region)
+    out_h = torch.empty(q_h.shape, dtype=torch.bfloat16, pin_memory=True)
+    for _ in range(2):
+        svg.sparse_attention(pb, q_h, k_h, v_h, gq_h, gk_h, si_h, buf, out_h)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        svg.sparse_attention(pb, q_h, k_h, v_h, gq_h, gk_h, si_h, buf, out_h)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, gq_h, gk_h, si_h))
+    d2h = out_h.numel() * out_h.element_size()
+
+    # ---- dense reference point on the same inputs (every head DENSE), outside the timed region
+    dense_ms = None
+    if not args.no_dense:
+        dk = torch.full_like(buf.kinds, svg.DENSE)
+        cap_d = svg.block_index_capacity(pb)
+        rp_d, col_d, full_d = svg.build_block_index(pb, dk, cap_d)
+        out_d = torch.empty_like(buf.qp)
+        svg.block_sparse_attn(pb, q, k, v, dk, rp_d, col_d, full_d, out=out_d)
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        svg.block_sparse_attn(pb, q, k, v, dk, rp_d, col_d, full_d, out=out_d)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = d0.elapsed_time(d1)
+        dense_flops = kept_tile_flops(rp_d.cpu().numpy(), col_d[: int(rp_d[-1])].cpu().numpy(), wl)
+        del out_d, rp_d, col_d, full_d
+    svg.sync_status()
+
+    # ---- max over ranks
+    vals = torch.tensor([total_ms, e2e_ms, stage_ms["attention"]], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms, attn_ms_max = (float(x) for x in vals.cpu())
+    ms_per_step = total_ms / args.steps
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    if rank != 0:
+        return None
+
+    pk, pk_src = peaks()
+    attn_tflops = flops / (stage_ms["attention"] * 1e-3) / 1e12
+    traffic = traffic_from_profile("attention.cuh", "attention_hunyuan_cfg3.md")
+    d, L, BH = wl.d, wl.L, wl.B * wl.H
+    stage_bytes = {"qknorm_rope": 8.0 * BH * L * d, "layout": 12.0 * BH * L * d, "inverse_layout": 4.0 * BH * L * d,
+                   "profile": 4.0 * BH * L * d}
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V with planted spatial/temporal heads; no model weights)",
+        "config": {
+            "workload": f"{wl.name} (HunyuanVideo 720p 5 s shape)",
+            "B": wl.B, "H": wl.H, "d": wl.d, "frames": wl.F, "grid": f"{wl.Hs}x{wl.Ws}", "text_tokens": wl.T,
+            "video_tokens": wl.Lv, "seq_len": wl.L, "spatial_window": wl.w, "temporal_radius": wl.r,
+            "tile": f"{wl.bq}x{wl.bk}", "profiled_rows": wl.n_samples,
+            "head_kinds": {"spatial": int((kinds == 0).sum()), "temporal": int((kinds == 1).sum())},
+            "kept_tile_tflop": round(flops / 1e12, 4),
+            "l2": "no flush: each step reads > 2 GB of inputs, far above the 126 MB L2",
+            "parallelism": f"replicas x{world} (one independent layer per GPU)",
+        },
+        "layer_ms": round(ms_per_step, 4),
+        "pct_bf16_peak": {"measured_sustained": round(100 * value / world / pk["bf16_tflops_sustained"], 2),
+                          "measured_burst": round(100 * value / world / pk["bf16_tflops"], 2),
+                          "nominal": round(100 * value / world / NOMINAL_BF16_TFLOPS, 2)},
+        "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+        "stage_gbs": {k: round(stage_bytes[k] / (stage_ms[k] * 1e-3) / 1e9, 1) for k in stage_bytes},
+        "roofline": {
+            "kernel": "attn_kernel<128> (svg_block_sparse_attn)",
+            "bound": "tensor",
+            "achieved": round(attn_tflops, 2),
+            "peak": pk["bf16_tflops_sustained"],
+            "unit": "TFLOP/s",
+            "frac": round(attn_tflops / pk["bf16_tflops_sustained"], 4),
+            "peak_source": f"{pk_src} bf16 sustained (kernel timed inside back-to-back steps)",
+            "frac_of_burst_peak": round(attn_tflops / pk["bf16_tflops"], 4),
+            "traffic": traffic,
+        },
+        "dense_attention": None if dense_ms is None else {
+            "ms": round(dense_ms, 3), "tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 2),
+            "speedup_sparse_attn_vs_dense": round(dense_ms / stage_ms["attention"], 3),
+            "theoretical_speedup_tiles": round(dense_flops / flops, 3)},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_rows)
+    return line
+
+
+# ---------------------------------------------------------- oracle (CPU) --
+
+def oracle_sample_rate(wl, n_rows: int, seed: int = 0):
+    """Times the fp64 oracle on a bounded sample of the step: QK-Norm+RoPE of
+    the sampled rows' Q and of K, and masked attention of `n_rows` query rows
+    spread over the heads (planted head kinds).  Returns (TFLOP/s counted like
+    the GPU metric, seconds, threads, description)."""
+    import oracle
+    inp = W.make_inputs(wl)
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    kinds = np.array([0 if c == "S" else 1 for c in wl.planted], np.uint8)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    per_head = max(1, n_rows // (wl.B * wl.H))
+    rows = np.concatenate([bh * wl.L + rng.choice(wl.L, per_head, replace=False) for bh in range(wl.B * wl.H)])
+    # the attention rows need normalised Q rows and every normalised K row of their heads
+    t0 = time.perf_counter()
+    qn_rows = oracle.qknorm_rope_f64(sh, pr, inp["q"], inp["gamma_q"], rows)
+    kn = oracle.qknorm_rope(sh, pr, inp["k"], inp["gamma_k"])
+    qn = np.zeros_like(inp["q"]).reshape(-1, wl.d)
+    qn[rows] = oracle.f64_to_bf16(qn_rows)
+    qn = qn.reshape(inp["q"].shape)
+    oracle.attention_rows(sh, pr, kinds, qn, kn, inp["v"], rows)
+    secs = time.perf_counter() - t0
+    # FLOPs the GPU metric would count for these rows: 4*d per (row, key column) of its kept tiles
+    flops = 0.0
+    cache = {}
+    for r in rows:
+        bh, tok = divmod(int(r), wl.L)
+        kind = int(kinds[bh])
+        qb = oracle.perm(sh, kind, tok) // wl.bq
+        if (kind, qb) not in cache:
+            cache[(kind, qb)] = kept_cols_closed(wl, kind, qb)
+        flops += 4.0 * wl.d * cache[(kind, qb)]
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    desc = (f"fp64 oracle: QK-Norm+RoPE of {len(rows)} Q rows and all K rows, masked attention of "
+            f"{len(rows)} query rows ({per_head} per head), FLOPs counted as kept-tile columns x 4d")
+    return flops / secs / 1e12, secs, threads, desc
+
+
+def kept_cols_closed(wl, kind, qb):
+    """Key columns of the tiles listed for one query tile (used only to count
+    the oracle sample's FLOPs at the largest shape)."""
+    L, Lv, S, F, bq, bk = wl.L, wl.Lv, wl.S, wl.F, wl.bq, wl.bk
+    r0, r1 = qb * bq, min(L, qb * bq + bq)
+    nkb = wl.nkb
+    if kind == 2 or r1 > Lv:
+        kbs = range(nkb)
+    else:
+        def iv(p):
+            if kind == 0:
+                f = p // S
+                return max(f - wl.w, 0) * S, min(f + wl.w + 1, F) * S
+            s = p // F
+            return max(s - wl.r, 0) * F, min(s + wl.r + 1, S) * F
+        lo, hi = iv(r0)[0], iv(r1 - 1)[1]
+        kbs = set(range(lo // bk, (hi - 1) // bk + 1))
+        if wl.T > 0:
+            kbs |= set(range(Lv // bk, nkb))
+    return int(sum(min(bk, L - kb * bk) for kb in kbs))
+
+
+def cpu_baseline(wl, n_rows):
+    rate, secs, threads, desc = oracle_sample_rate(wl, n_rows)
+    return {"value": round(rate, 8), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": desc, "seconds": round(secs, 2)}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    wl = W.CONFIGS[args.config]
+    rates, secs_all = [], []
+    for s in range(args.warmup + args.steps):
+        rate, secs, threads, desc = oracle_sample_rate(wl, args.ref_rows, seed=s)
+        if s >= args.warmup:
+            rates.append(rate)
+            secs_all.append(secs)
+    value = statistics.mean(rates)
+    flops_step = value * 1e12 * statistics.mean(secs_all)
+    return {
+        "metric": METRIC, "value": round(value, 8), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1000 * statistics.mean(secs_all), 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{wl.name} (HunyuanVideo 720p 5 s shape)", "B": wl.B, "H": wl.H, "d": wl.d,
+                   "seq_len": wl.L, "sampled_rows_per_step": args.ref_rows,
+                   "kept_tile_gflop_per_step": round(flops_step / 1e9, 3)},
+        "cpu_baseline": {"value": round(value, 8), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 8), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------- main --
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--config", type=int, default=3)
+    ap.add_argument("--cpu-rows", type=int, default=480)
+    ap.add_argument("--ref-rows", type=int, default=240)
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if world != args.gpus:
+        world = max(world, 1)
+    if args.impl == "reference":
+        line = run_reference(args, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

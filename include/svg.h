@@ -1,0 +1,204 @@
+/*
+ * svg.h — C ABI of the B200 (sm_100a) Sparse VideoGen attention step.
+ *
+ * The step, as the pages describe it (page title, section):
+ *   1. QK-Norm (RMSNorm) and 3D RoPE on Q and K
+ *        ("Sparse VideoGen" WeChat article, "其他优化方法";
+ *         ICML 2025 report (机器之心), "Layout Transformation + Kernel 加速");
+ *   2. online profiling: a few sampled query rows per head are attended densely,
+ *      with the spatial mask and with the temporal mask; each head takes the mask
+ *      with the smaller MSE against dense
+ *        (article, "Online Profiling Strategy"; report, "动态自适应的稀疏策略" steps 1-3);
+ *   3. frame-major -> token-major layout transform for temporal heads
+ *        (article, "硬件高效的 Layout Transformation"; report, "Layout Transformation + Kernel 加速");
+ *   4. per-head block-sparse attention over the kept key tiles
+ *        (article, "Spatial Head" / "Temporal Head" / "其他优化方法"; report, "Sparse VideoGen 的核心设计");
+ *   5. the inverse layout transform of the output.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors Q, K, V, O are bfloat16 (passed as uint16_t bit patterns), contiguous
+ *     [B, H, L, d] with d in {64, 128}; L = F*Hs*Ws + text_len.  Video token
+ *     i < F*Hs*Ws is frame f = i / (Hs*Ws), spatial index s = i % (Hs*Ws),
+ *     grid position (s / Ws, s % Ws).  Text tokens follow the video tokens.
+ *   - "device" pointers are CUDA device memory owned by the caller; every device
+ *     pointer must be 16-byte aligned.  "host" pointers are ordinary host memory.
+ *     The library never frees or keeps caller memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Kernels are
+ *     enqueued on it; calls return without synchronising.
+ *   - Argument errors are detected on the host before anything is enqueued and
+ *     returned as a status; nothing is launched then.  A launch failure returns
+ *     SVG_ERR_CUDA.  Errors found by the kernels themselves (a bounded wait that
+ *     ran out, a block list larger than its capacity) are recorded in a per-device
+ *     error word that svg_sync_status() reads and clears.
+ *   - Outputs never alias inputs.
+ */
+#ifndef SVG_H
+#define SVG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVG_OK = 0,
+  SVG_ERR_INVALID_ARG = 1,   /* null pointer, bad flag, n out of range            */
+  SVG_ERR_SHAPE = 2,         /* inconsistent shape (L != F*Hs*Ws + text_len, ...)  */
+  SVG_ERR_UNSUPPORTED = 3,   /* valid but not implemented (d, tile sizes, split)    */
+  SVG_ERR_ALIGNMENT = 4,     /* a device pointer is not 16-byte aligned             */
+  SVG_ERR_CAPACITY = 5,      /* a caller buffer is too small                        */
+  SVG_ERR_CUDA = 6,          /* a CUDA call or launch failed                        */
+  SVG_ERR_TIMEOUT = 7        /* a kernel's bounded wait ran out (device error word) */
+} svg_status;
+
+typedef enum {
+  SVG_HEAD_SPATIAL = 0,      /* keys whose frame is within +-spatial_frames        */
+  SVG_HEAD_TEMPORAL = 1,     /* keys whose spatial index is within +-temporal_radius */
+  SVG_HEAD_DENSE = 2         /* every key                                           */
+} svg_head_kind;
+
+typedef struct {
+  int B, H;                  /* batch, heads                                         */
+  int L;                     /* sequence length = F*Hs*Ws + text_len                 */
+  int d;                     /* head dimension: 64 or 128                            */
+  int F, Hs, Ws;             /* latent frames and per-frame spatial grid             */
+  int text_len;              /* text tokens after the video tokens (always kept)     */
+} svg_shape;
+
+typedef struct {
+  int spatial_frames;        /* w: spatial head keeps |frame_q - frame_k| <= w        */
+  int temporal_radius;       /* r: temporal head keeps |s_q - s_k| <= r               */
+  int block_q;               /* query tile rows of the block list: 64 or 128          */
+  int block_k;               /* key tile columns of the block list: 64               */
+  float eps;                 /* RMSNorm epsilon                                      */
+  float rope_base;           /* RoPE base (e.g. 10000)                               */
+  int rope_split[3];         /* RoPE widths of the t, h, w sections; even; sum = d    */
+  float softmax_scale;       /* 0 -> 1/sqrt(d)                                        */
+} svg_params;
+
+enum { SVG_NORM_ROPE = 1, SVG_LAYOUT = 2 };
+
+/* ------------------------------------------------------------------------ */
+/* Stage 1 (+3): QK-Norm + 3D RoPE and/or the layout transform.
+ *   flags & SVG_NORM_ROPE: q_out/k_out rows = RMSNorm(row) * gamma, then, on video
+ *     rows only, RoPE: in section a (t, h, w; widths rope_split, laid out from d=0)
+ *     the pair (2j, 2j+1) is rotated by p_a * rope_base^(-2j/n_a), p_a = (f, y, x).
+ *     Arithmetic in fp32; results rounded to nearest-even bf16.
+ *   flags & SVG_LAYOUT: rows are written in the head's layout: for heads whose
+ *     head_kind is TEMPORAL, video row f*S+s goes to s*F+f (S = Hs*Ws); text rows and
+ *     other heads stay in place.  v (required with LAYOUT) is moved the same way
+ *     without normalisation.
+ * q, k, v, q_out, k_out, v_out: device bf16 [B,H,L,d].  v/v_out are used only with
+ *   SVG_LAYOUT (may be NULL otherwise).
+ * gamma_q, gamma_k: device fp32 [d]; required with SVG_NORM_ROPE.
+ * rope_table: device fp32 table of svg_rope_table_size() floats written on the host
+ *   by svg_rope_table_fill() and copied by the caller; required with SVG_NORM_ROPE.
+ * head_kind: device uint8 [B*H]; required with SVG_LAYOUT. */
+svg_status svg_qknorm_rope_layout(const svg_shape* shape, const svg_params* params, int flags,
+                                  const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                  const float* gamma_q, const float* gamma_k, const float* rope_table,
+                                  const uint8_t* head_kind,
+                                  uint16_t* q_out, uint16_t* k_out, uint16_t* v_out, void* stream);
+
+/* Stage 2: online profiling.
+ * For every (b, h) and each of the n sampled video tokens sample_idx[0..n) (device
+ * int32, the same rows for every head, 1 <= n <= 64): the dense, the spatial-masked and
+ * the temporal-masked attention outputs of that query row (fp32 softmax, P split into
+ * two bf16 terms for the tensor-core products).  Per head
+ *   MSE_m = mean over the n rows and d columns of (O_m - O_dense)^2,  m in {spatial, temporal}
+ * and head_kind_out[b*H+h] = SPATIAL if MSE_spatial <= MSE_temporal else TEMPORAL.
+ * qn, kn: device bf16 [B,H,L,d] after stage 1, frame-major order; v: device bf16.
+ * workspace: device scratch of at least svg_profile_workspace_size(shape, n) bytes.
+ * mse_out: device fp32 [B*H*2] (spatial, temporal) or NULL.
+ * head_kind_out: device uint8 [B*H]. */
+svg_status svg_profile_heads(const svg_shape* shape, const svg_params* params,
+                             const uint16_t* qn, const uint16_t* kn, const uint16_t* v,
+                             const int32_t* sample_idx, int n, void* workspace, size_t workspace_bytes,
+                             float* mse_out, uint8_t* head_kind_out, void* stream);
+
+/* Block index (not on the pages; the block-sparse kernel they describe needs it).
+ * In each head's layout, the tile (q-block qb: rows [qb*block_q, +block_q),
+ * k-block kb: keys [kb*block_k, +block_k), rows/keys >= L excluded) is listed iff at
+ * least one (query, key) pair in it is kept by the head's mask; full[e] = 1 iff every
+ * pair is kept.  CSR over (b, h, qb) in that order, kb ascending:
+ *   row_ptr: device int32 [B*H*nqb + 1], col: device int32 [capacity],
+ *   full: device uint8 [capacity].
+ * If the list needs more than `capacity` entries, nothing past capacity is written
+ * and svg_sync_status() reports SVG_ERR_CAPACITY.  svg_block_index_capacity() is
+ * always enough. */
+svg_status svg_build_block_index(const svg_shape* shape, const svg_params* params,
+                                 const uint8_t* head_kind, int32_t* row_ptr, int32_t* col,
+                                 uint8_t* full, int64_t capacity, void* stream);
+
+/* Stage 4: block-sparse attention, tcgen05/TMEM tile loop fed by TMA.
+ *   out[b,h,i,:] = sum_k softmax_k(scale * q_i . k_k | kept) v_k
+ * over the keys of the tiles listed for the query's q-block, with the head's
+ * token-level mask applied inside partial tiles (full = 0) and to keys >= L.
+ * Online softmax in fp32; P rounded to bf16 for the P.V product.
+ * q, k, v: device bf16 [B,H,L,d] in the head's layout (stage 3 output).
+ * head_kind: device uint8 [B*H].  row_ptr/col/full: the block index above.
+ * out: device bf16 [B,H,L,d] in the head's layout.
+ * lse_out: device fp32 [B,H,L] natural-log sum of exp of the kept scaled logits, or NULL.
+ * Requires block_k = 64 and block_q in {64, 128}. */
+svg_status svg_block_sparse_attn(const svg_shape* shape, const svg_params* params,
+                                 const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                 const uint8_t* head_kind, const int32_t* row_ptr,
+                                 const int32_t* col, const uint8_t* full,
+                                 uint16_t* out, float* lse_out, void* stream);
+
+/* Stage 5: inverse of the layout transform (temporal heads: row s*F+f -> f*S+s).
+ * src, dst: device bf16 [B,H,L,d]; head_kind: device uint8 [B*H]. */
+svg_status svg_inverse_layout(const svg_shape* shape, const uint8_t* head_kind,
+                              const uint16_t* src, uint16_t* dst, void* stream);
+
+/* The five stages in order on one stream (profiling skipped when
+ * head_kind_in != NULL, whose kinds are then used).  All buffers are device
+ * memory owned by the caller:
+ *   qn, kn, qp, kp, vp: bf16 [B,H,L,d] intermediates; op: bf16 [B,H,L,d] output
+ *   in the head's layout; out: bf16 [B,H,L,d] final output in model order;
+ *   head_kind_out: uint8 [B*H]; mse_out: fp32 [B*H*2] or NULL;
+ *   row_ptr/col/full: block index with `capacity` entries;
+ *   workspace: svg_profile_workspace_size(shape, n) bytes. */
+svg_status svg_attention_step(const svg_shape* shape, const svg_params* params,
+                              const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                              const float* gamma_q, const float* gamma_k, const float* rope_table,
+                              const int32_t* sample_idx, int n, const uint8_t* head_kind_in,
+                              uint16_t* qn, uint16_t* kn, uint16_t* qp, uint16_t* kp, uint16_t* vp,
+                              uint16_t* op, uint16_t* out, uint8_t* head_kind_out, float* mse_out,
+                              int32_t* row_ptr, int32_t* col, uint8_t* full, int64_t capacity,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* ----------------------------------------------------------- host helpers */
+
+/* n distinct video-token indices in [0, Lv) into host_out[0..n): the first n slots of
+ * a partial Fisher-Yates shuffle driven by SplitMix64(seed) (slot i swaps with
+ * i + x mod (Lv - i)).  Host only; needs no GPU. */
+svg_status svg_sample_queries(uint64_t seed, int64_t Lv, int n, int32_t* host_out);
+
+/* Number of fp32 values of the RoPE table, and its contents (host memory):
+ * for section a, position p in [0, F | Hs | Ws), pair j < n_a/2: (cos, sin) of
+ * p * base^(-2j/n_a), computed in double and rounded to float. */
+size_t svg_rope_table_size(const svg_shape* shape, const svg_params* params);
+svg_status svg_rope_table_fill(const svg_shape* shape, const svg_params* params, float* host_out);
+
+/* Entries that always suffice for svg_build_block_index: B*H*nqb*nkb. */
+int64_t svg_block_index_capacity(const svg_shape* shape, const svg_params* params);
+
+/* Device scratch bytes svg_profile_heads needs for n sampled rows. */
+size_t svg_profile_workspace_size(const svg_shape* shape, int n);
+
+/* Synchronises `stream`, then reads and clears this device's error word:
+ * SVG_OK, SVG_ERR_TIMEOUT or SVG_ERR_CAPACITY (or SVG_ERR_CUDA if the
+ * synchronisation itself failed). */
+svg_status svg_sync_status(void* stream);
+
+const char* svg_status_string(svg_status status);
+const char* svg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVG_H */

@@ -1,0 +1,260 @@
+"""Python binding of the C ABI (include/svg.h).
+
+Argument marshalling only: torch tensors are passed to the library as raw
+device pointers on the current CUDA stream; every stage runs in the library's
+sm_100a kernels.  PyTorch provides device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import _lib as C
+from ._lib import check, lib
+
+SPATIAL, TEMPORAL, DENSE = C.SVG_HEAD_SPATIAL, C.SVG_HEAD_TEMPORAL, C.SVG_HEAD_DENSE
+
+
+@dataclass(frozen=True)
+class Problem:
+    """Shape and mask parameters of one attention layer (see svg_shape / svg_params)."""
+    B: int
+    H: int
+    d: int
+    F: int
+    Hs: int
+    Ws: int
+    text_len: int
+    spatial_frames: int
+    temporal_radius: int
+    block_q: int = 128
+    block_k: int = 64
+    eps: float = 1e-6
+    rope_base: float = 10000.0
+    rope_split: tuple = None
+    softmax_scale: float = 0.0
+
+    @property
+    def S(self):
+        return self.Hs * self.Ws
+
+    @property
+    def Lv(self):
+        return self.F * self.S
+
+    @property
+    def L(self):
+        return self.Lv + self.text_len
+
+    @property
+    def nqb(self):
+        return -(-self.L // self.block_q)
+
+    @property
+    def nkb(self):
+        return -(-self.L // self.block_k)
+
+    @classmethod
+    def from_workload(cls, wl, **over):
+        kw = dict(B=wl.B, H=wl.H, d=wl.d, F=wl.F, Hs=wl.Hs, Ws=wl.Ws, text_len=wl.T,
+                  spatial_frames=wl.w, temporal_radius=wl.r, block_q=wl.bq, block_k=wl.bk,
+                  eps=wl.eps, rope_base=wl.rope_base, rope_split=tuple(wl.rope_split))
+        kw.update(over)
+        return cls(**kw)
+
+    def c_shape(self) -> C.SvgShape:
+        return C.SvgShape(self.B, self.H, self.L, self.d, self.F, self.Hs, self.Ws, self.text_len)
+
+    def c_params(self) -> C.SvgParams:
+        split = self.rope_split or (self.d // 4, 3 * self.d // 8, 3 * self.d // 8)
+        return C.SvgParams(self.spatial_frames, self.temporal_radius, self.block_q, self.block_k,
+                           self.eps, self.rope_base, (ctypes.c_int * 3)(*split), self.softmax_scale)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _empty_like_bf16(x):
+    return torch.empty_like(x)
+
+
+# ------------------------------------------------------------ host helpers --
+
+def sample_queries(seed: int, Lv: int, n: int) -> np.ndarray:
+    out = np.empty(n, np.int32)
+    check(lib().svg_sample_queries(seed, Lv, n, out.ctypes.data), "svg_sample_queries")
+    return out
+
+
+def rope_table(pb: Problem) -> np.ndarray:
+    sh, pr = pb.c_shape(), pb.c_params()
+    n = lib().svg_rope_table_size(ctypes.byref(sh), ctypes.byref(pr))
+    out = np.empty(n, np.float32)
+    check(lib().svg_rope_table_fill(ctypes.byref(sh), ctypes.byref(pr), out.ctypes.data), "svg_rope_table_fill")
+    return out
+
+
+def block_index_capacity(pb: Problem) -> int:
+    sh, pr = pb.c_shape(), pb.c_params()
+    return int(lib().svg_block_index_capacity(ctypes.byref(sh), ctypes.byref(pr)))
+
+
+def profile_workspace_size(pb: Problem, n: int) -> int:
+    sh = pb.c_shape()
+    return int(lib().svg_profile_workspace_size(ctypes.byref(sh), n))
+
+
+def sync_status(stream=None):
+    """Synchronise the stream and raise if a kernel reported an error."""
+    check(lib().svg_sync_status(_stream(stream)), "svg_sync_status")
+
+
+# ------------------------------------------------------------------ stages --
+
+def qknorm_rope_layout(pb: Problem, q, k, v=None, gamma_q=None, gamma_k=None, table=None, kinds=None,
+                       flags=C.SVG_NORM_ROPE, out=None, stream=None):
+    """Stage 1 (flags has NORM_ROPE) and/or stage 3 (flags has LAYOUT).
+    Returns (q_out, k_out, v_out or None)."""
+    sh, pr = pb.c_shape(), pb.c_params()
+    if out is None:
+        out = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v) if (flags & C.SVG_LAYOUT) else None)
+    qo, ko, vo = out
+    st = lib().svg_qknorm_rope_layout(ctypes.byref(sh), ctypes.byref(pr), flags, _p(q), _p(k), _p(v),
+                                      _p(gamma_q), _p(gamma_k), _p(table), _p(kinds), _p(qo), _p(ko), _p(vo),
+                                      _stream(stream))
+    check(st, "svg_qknorm_rope_layout")
+    return qo, ko, vo
+
+
+def qknorm_rope(pb: Problem, q, k, gamma_q, gamma_k, table, out=None, stream=None):
+    qo, ko, _ = qknorm_rope_layout(pb, q, k, None, gamma_q, gamma_k, table, None, C.SVG_NORM_ROPE,
+                                   None if out is None else (out[0], out[1], None), stream)
+    return qo, ko
+
+
+def layout(pb: Problem, q, k, v, kinds, out=None, stream=None):
+    return qknorm_rope_layout(pb, q, k, v, None, None, None, kinds, C.SVG_LAYOUT, out, stream)
+
+
+def profile_heads(pb: Problem, qn, kn, v, sample_idx, workspace=None, kinds_out=None, mse_out=None, stream=None):
+    """Returns (kinds uint8 [B*H], mse fp32 [B*H, 2])."""
+    sh, pr = pb.c_shape(), pb.c_params()
+    n = int(sample_idx.numel())
+    need = profile_workspace_size(pb, n)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=qn.device)
+    if kinds_out is None:
+        kinds_out = torch.empty(pb.B * pb.H, dtype=torch.uint8, device=qn.device)
+    if mse_out is None:
+        mse_out = torch.empty(pb.B * pb.H, 2, dtype=torch.float32, device=qn.device)
+    st = lib().svg_profile_heads(ctypes.byref(sh), ctypes.byref(pr), _p(qn), _p(kn), _p(v), _p(sample_idx), n,
+                                 _p(workspace), workspace.numel() * workspace.element_size(), _p(mse_out),
+                                 _p(kinds_out), _stream(stream))
+    check(st, "svg_profile_heads")
+    return kinds_out, mse_out
+
+
+def build_block_index(pb: Problem, kinds, capacity=None, out=None, stream=None):
+    """Returns (row_ptr int32 [B*H*nqb+1], col int32 [capacity], full uint8 [capacity]).
+    Only the first row_ptr[-1] entries of col/full are meaningful."""
+    sh, pr = pb.c_shape(), pb.c_params()
+    if capacity is None:
+        capacity = block_index_capacity(pb)
+    dev = kinds.device
+    if out is None:
+        out = (torch.empty(pb.B * pb.H * pb.nqb + 1, dtype=torch.int32, device=dev),
+               torch.empty(capacity, dtype=torch.int32, device=dev),
+               torch.empty(capacity, dtype=torch.uint8, device=dev))
+    row_ptr, col, full = out
+    st = lib().svg_build_block_index(ctypes.byref(sh), ctypes.byref(pr), _p(kinds), _p(row_ptr), _p(col), _p(full),
+                                     capacity, _stream(stream))
+    check(st, "svg_build_block_index")
+    return row_ptr, col, full
+
+
+def block_sparse_attn(pb: Problem, q, k, v, kinds, row_ptr, col, full, out=None, want_lse=False, stream=None):
+    sh, pr = pb.c_shape(), pb.c_params()
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty(pb.B, pb.H, pb.L, dtype=torch.float32, device=q.device) if want_lse else None
+    st = lib().svg_block_sparse_attn(ctypes.byref(sh), ctypes.byref(pr), _p(q), _p(k), _p(v), _p(kinds),
+                                     _p(row_ptr), _p(col), _p(full), _p(out), _p(lse), _stream(stream))
+    check(st, "svg_block_sparse_attn")
+    return (out, lse) if want_lse else out
+
+
+def inverse_layout(pb: Problem, kinds, src, out=None, stream=None):
+    sh = pb.c_shape()
+    if out is None:
+        out = torch.empty_like(src)
+    st = lib().svg_inverse_layout(ctypes.byref(sh), _p(kinds), _p(src), _p(out), _stream(stream))
+    check(st, "svg_inverse_layout")
+    return out
+
+
+# --------------------------------------------------------------- full step --
+
+class StepBuffers:
+    """Device buffers of one step, allocated once for a Problem and reused."""
+
+    def __init__(self, pb: Problem, n_samples: int, device="cuda"):
+        shp = (pb.B, pb.H, pb.L, pb.d)
+        mk = lambda: torch.empty(shp, dtype=torch.bfloat16, device=device)
+        self.pb = pb
+        self.n = n_samples
+        self.qn, self.kn, self.qp, self.kp, self.vp, self.op, self.out = (mk() for _ in range(7))
+        self.kinds = torch.empty(pb.B * pb.H, dtype=torch.uint8, device=device)
+        self.mse = torch.empty(pb.B * pb.H, 2, dtype=torch.float32, device=device)
+        self.capacity = block_index_capacity(pb)
+        self.row_ptr = torch.empty(pb.B * pb.H * pb.nqb + 1, dtype=torch.int32, device=device)
+        self.col = torch.empty(self.capacity, dtype=torch.int32, device=device)
+        self.full = torch.empty(self.capacity, dtype=torch.uint8, device=device)
+        self.workspace = torch.empty(max(profile_workspace_size(pb, n_samples), 16), dtype=torch.uint8,
+                                     device=device)
+        self.table = torch.from_numpy(rope_table(pb)).to(device)
+
+
+def attention_step(pb: Problem, q, k, v, gamma_q, gamma_k, sample_idx, buffers: StepBuffers,
+                   kinds_in=None, stream=None):
+    """All five stages on device tensors through svg_attention_step; returns
+    buffers.out (model order).  With kinds_in the profiling stage is skipped."""
+    b = buffers
+    sh, pr = pb.c_shape(), pb.c_params()
+    st = lib().svg_attention_step(
+        ctypes.byref(sh), ctypes.byref(pr), _p(q), _p(k), _p(v), _p(gamma_q), _p(gamma_k), _p(b.table),
+        _p(sample_idx), int(sample_idx.numel()), _p(kinds_in), _p(b.qn), _p(b.kn), _p(b.qp), _p(b.kp), _p(b.vp),
+        _p(b.op), _p(b.out), _p(b.kinds), _p(b.mse), _p(b.row_ptr), _p(b.col), _p(b.full), b.capacity,
+        _p(b.workspace), b.workspace.numel(), _stream(stream))
+    check(st, "svg_attention_step")
+    return b.out
+
+
+def sparse_attention(pb: Problem, q_host, k_host, v_host, gamma_q, gamma_k, sample_idx, buffers: StepBuffers = None,
+                     out_host=None, device="cuda", stream=None):
+    """End-to-end call on host tensors: copies Q/K/V (bf16 [B,H,L,d], pinned for
+    asynchronous copies), gamma and the sample in, runs the step, copies O back
+    into `out_host` (allocated pinned if None).  Returns out_host."""
+    if buffers is None:
+        buffers = StepBuffers(pb, int(sample_idx.numel()), device)
+    s = stream if stream is not None else torch.cuda.current_stream()
+    with torch.cuda.stream(s):
+        q = q_host.to(device, non_blocking=True)
+        k = k_host.to(device, non_blocking=True)
+        v = v_host.to(device, non_blocking=True)
+        gq = gamma_q.to(device, non_blocking=True)
+        gk = gamma_k.to(device, non_blocking=True)
+        si = sample_idx.to(device, non_blocking=True)
+        o = attention_step(pb, q, k, v, gq, gk, si, buffers, stream=s)
+        if out_host is None:
+            out_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        out_host.copy_(o, non_blocking=True)
+    return out_host

@@ -1,0 +1,439 @@
+// svg_lib.cu — the C ABI declared in include/svg.h: host-side argument
+// checks, launch geometry, TMA tensor maps, and the host helpers.  All
+// kernels are in the included .cuh files (one translation unit).
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "attention.cuh"
+#include "block_index.cuh"
+#include "profile.cuh"
+#include "rowmap.cuh"
+#include "svg_common.cuh"
+
+using namespace svg;
+
+namespace {
+
+constexpr int kNumSMs = 148;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+svg_status check_shape(const svg_shape* s) {
+  if (!s) return SVG_ERR_INVALID_ARG;
+  if (s->B <= 0 || s->H <= 0 || s->F <= 0 || s->Hs <= 0 || s->Ws <= 0 || s->text_len < 0) return SVG_ERR_SHAPE;
+  const long long Lv = static_cast<long long>(s->F) * s->Hs * s->Ws;
+  if (Lv + s->text_len != s->L) return SVG_ERR_SHAPE;
+  if (s->L >= (1 << 30)) return SVG_ERR_UNSUPPORTED;
+  if (s->d != 64 && s->d != 128) return SVG_ERR_UNSUPPORTED;
+  if (static_cast<long long>(s->B) * s->H > (1 << 24)) return SVG_ERR_UNSUPPORTED;
+  return SVG_OK;
+}
+
+svg_status check_params(const svg_shape* s, const svg_params* p, bool need_tiles) {
+  if (!p) return SVG_ERR_INVALID_ARG;
+  if (p->spatial_frames < 0 || p->temporal_radius < 0) return SVG_ERR_INVALID_ARG;
+  if (need_tiles) {
+    if (p->block_k != 64) return SVG_ERR_UNSUPPORTED;
+    if (p->block_q != 64 && p->block_q != 128) return SVG_ERR_UNSUPPORTED;
+  }
+  if (!(p->eps >= 0.f) || !(p->softmax_scale >= 0.f)) return SVG_ERR_INVALID_ARG;
+  (void)s;
+  return SVG_OK;
+}
+
+svg_status check_rope(const svg_shape* s, const svg_params* p) {
+  const int* sp = p->rope_split;
+  if (sp[0] < 0 || sp[1] < 0 || sp[2] < 0) return SVG_ERR_INVALID_ARG;
+  if ((sp[0] | sp[1] | sp[2]) & 1) return SVG_ERR_UNSUPPORTED;
+  if (sp[0] + sp[1] + sp[2] != s->d) return SVG_ERR_SHAPE;
+  if (!(p->rope_base > 0.f)) return SVG_ERR_INVALID_ARG;
+  return SVG_OK;
+}
+
+Geometry make_geometry(const svg_shape* s, const svg_params* p) {
+  Geometry g{};
+  g.B = s->B;
+  g.H = s->H;
+  g.L = s->L;
+  g.d = s->d;
+  g.F = s->F;
+  g.Hs = s->Hs;
+  g.Ws = s->Ws;
+  g.T = s->text_len;
+  g.S = s->Hs * s->Ws;
+  g.Lv = g.F * g.S;
+  g.BH = s->B * s->H;
+  if (p) {
+    g.w = p->spatial_frames;
+    g.r = p->temporal_radius;
+    g.bq = p->block_q > 0 ? p->block_q : 128;
+    g.bk = p->block_k > 0 ? p->block_k : 64;
+  } else {
+    g.bq = 128;
+    g.bk = 64;
+  }
+  g.nqb = (g.L + g.bq - 1) / g.bq;
+  g.nkb = (g.L + g.bk - 1) / g.bk;
+  return g;
+}
+
+float scale_of(const svg_shape* s, const svg_params* p) {
+  return (p->softmax_scale > 0.f) ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(s->d));
+}
+
+svg_status launch_status() {
+  return (cudaGetLastError() == cudaSuccess) ? SVG_OK : SVG_ERR_CUDA;
+}
+
+// ----------------------------------------------------------- tensor maps --
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D map over a [BH, L, D] bf16 tensor: dims (D, L, BH), box (64, rows, 1),
+// 128-byte swizzle; rows past L read as zero.
+bool make_map(CUtensorMap* m, const void* base, int D, int L, int BH, int rows) {
+  auto enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+// ------------------------------------------------------------- rowmap ----
+
+svg_status launch_rowmap(const RowmapArgs& a, int D, cudaStream_t st) {
+  const int64_t rows = static_cast<int64_t>(a.g.BH) * a.g.L * a.ntensor;
+  const int rows_per_block = 8 * (32 / (D / 8)) * 4;   // warps * rows per step * steps
+  int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
+  if (blocks > kNumSMs * 8) blocks = kNumSMs * 8;
+  if (blocks < 1) blocks = 1;
+  if (D == 128)
+    rowmap_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
+  else
+    rowmap_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
+  return launch_status();
+}
+
+}  // namespace
+
+// ===================================================================== ABI
+
+extern "C" {
+
+const char* svg_version(void) { return "svg-b200 0.1 (sm_100a)"; }
+
+const char* svg_status_string(svg_status s) {
+  switch (s) {
+    case SVG_OK: return "ok";
+    case SVG_ERR_INVALID_ARG: return "invalid argument";
+    case SVG_ERR_SHAPE: return "inconsistent shape";
+    case SVG_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SVG_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case SVG_ERR_CAPACITY: return "buffer too small";
+    case SVG_ERR_CUDA: return "CUDA error";
+    case SVG_ERR_TIMEOUT: return "kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+svg_status svg_sample_queries(uint64_t seed, int64_t Lv, int n, int32_t* host_out) {
+  if (!host_out || n <= 0 || Lv <= 0 || n > Lv || Lv > INT32_MAX) return SVG_ERR_INVALID_ARG;
+  // partial Fisher-Yates over 0..Lv-1; only the touched slots are remembered
+  struct Slot { int64_t key, val; };
+  const int cap = 4 * n + 8;
+  Slot* tab = new Slot[cap];
+  int used = 0;
+  auto get = [&](int64_t key) -> int64_t {
+    for (int i = 0; i < used; i++)
+      if (tab[i].key == key) return tab[i].val;
+    return key;
+  };
+  auto put = [&](int64_t key, int64_t val) {
+    for (int i = 0; i < used; i++)
+      if (tab[i].key == key) {
+        tab[i].val = val;
+        return;
+      }
+    tab[used].key = key;
+    tab[used].val = val;
+    used++;
+  };
+  uint64_t state = seed;
+  for (int i = 0; i < n; i++) {
+    state += 0x9E3779B97F4A7C15ull;            // SplitMix64 (Steele, Lea, Flood 2014)
+    uint64_t z = state;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    z ^= z >> 31;
+    const int64_t j = i + static_cast<int64_t>(z % static_cast<uint64_t>(Lv - i));
+    const int64_t vi = get(i), vj = get(j);
+    put(i, vj);
+    put(j, vi);
+    host_out[i] = static_cast<int32_t>(vj);
+  }
+  delete[] tab;
+  return SVG_OK;
+}
+
+size_t svg_rope_table_size(const svg_shape* s, const svg_params* p) {
+  if (!s || !p) return 0;
+  return 2 * (static_cast<size_t>(s->F) * (p->rope_split[0] / 2) + static_cast<size_t>(s->Hs) * (p->rope_split[1] / 2) +
+              static_cast<size_t>(s->Ws) * (p->rope_split[2] / 2));
+}
+
+svg_status svg_rope_table_fill(const svg_shape* s, const svg_params* p, float* host_out) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if (!p || !host_out) return SVG_ERR_INVALID_ARG;
+  if ((st = check_rope(s, p)) != SVG_OK) return st;
+  const int npos[3] = {s->F, s->Hs, s->Ws};
+  size_t o = 0;
+  for (int a = 0; a < 3; a++) {
+    const int n = p->rope_split[a];
+    for (int pos = 0; pos < npos[a]; pos++) {
+      for (int j = 0; j < n / 2; j++) {
+        const double th = static_cast<double>(pos) * std::pow(static_cast<double>(p->rope_base), -2.0 * j / n);
+        host_out[o++] = static_cast<float>(std::cos(th));
+        host_out[o++] = static_cast<float>(std::sin(th));
+      }
+    }
+  }
+  return SVG_OK;
+}
+
+int64_t svg_block_index_capacity(const svg_shape* s, const svg_params* p) {
+  if (check_shape(s) != SVG_OK || !p || p->block_q <= 0 || p->block_k <= 0) return -1;
+  const int64_t nqb = (s->L + p->block_q - 1) / p->block_q, nkb = (s->L + p->block_k - 1) / p->block_k;
+  return static_cast<int64_t>(s->B) * s->H * nqb * nkb;
+}
+
+size_t svg_profile_workspace_size(const svg_shape* s, int n) {
+  if (check_shape(s) != SVG_OK || n <= 0) return 0;
+  const int BH = s->B * s->H;
+  const int nchunk = prof_chunks(BH, s->L);
+  return static_cast<size_t>(BH) * nchunk * kProfRows * prof_rec_floats(s->d) * sizeof(float);
+}
+
+svg_status svg_sync_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SVG_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(int)) != cudaSuccess) return SVG_ERR_CUDA;
+  const int zero = 0;
+  if (v && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return SVG_ERR_CUDA;
+  if (v & kErrTimeout) return SVG_ERR_TIMEOUT;
+  if (v & kErrCapacity) return SVG_ERR_CAPACITY;
+  if (v & kErrBadIndex) return SVG_ERR_INVALID_ARG;
+  return SVG_OK;
+}
+
+svg_status svg_qknorm_rope_layout(const svg_shape* s, const svg_params* p, int flags, const uint16_t* q,
+                                  const uint16_t* k, const uint16_t* v, const float* gamma_q, const float* gamma_k,
+                                  const float* rope_table, const uint8_t* head_kind, uint16_t* q_out,
+                                  uint16_t* k_out, uint16_t* v_out, void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if (!p) return SVG_ERR_INVALID_ARG;
+  if ((st = check_params(s, p, false)) != SVG_OK) return st;
+  if (flags == 0 || (flags & ~(SVG_NORM_ROPE | SVG_LAYOUT))) return SVG_ERR_INVALID_ARG;
+  if (!q || !k || !q_out || !k_out) return SVG_ERR_INVALID_ARG;
+  if (flags & SVG_NORM_ROPE) {
+    if (!gamma_q || !gamma_k || !rope_table) return SVG_ERR_INVALID_ARG;
+    if ((st = check_rope(s, p)) != SVG_OK) return st;
+  }
+  if (flags & SVG_LAYOUT) {
+    if (!v || !v_out || !head_kind) return SVG_ERR_INVALID_ARG;
+  }
+  const void* ptrs[] = {q, k, v, q_out, k_out, v_out, gamma_q, gamma_k, rope_table};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return SVG_ERR_ALIGNMENT;
+  if (q == q_out || k == k_out || (v && v == v_out)) return SVG_ERR_INVALID_ARG;
+  RowmapArgs a{};
+  a.g = make_geometry(s, p);
+  a.flags = flags;
+  a.ntensor = (flags & SVG_LAYOUT) ? 3 : 2;
+  a.norm_tensors = (flags & SVG_NORM_ROPE) ? 2 : 0;
+  a.src[0] = q;
+  a.src[1] = k;
+  a.src[2] = v;
+  a.dst[0] = q_out;
+  a.dst[1] = k_out;
+  a.dst[2] = v_out;
+  a.gamma[0] = gamma_q;
+  a.gamma[1] = gamma_k;
+  a.rope = reinterpret_cast<const float2*>(rope_table);
+  a.kind = head_kind;
+  a.eps = p->eps;
+  a.split0 = p->rope_split[0];
+  a.split1 = p->rope_split[1];
+  a.rope_off1 = s->F * (p->rope_split[0] / 2);
+  a.rope_off2 = a.rope_off1 + s->Hs * (p->rope_split[1] / 2);
+  return launch_rowmap(a, s->d, static_cast<cudaStream_t>(stream));
+}
+
+svg_status svg_inverse_layout(const svg_shape* s, const uint8_t* head_kind, const uint16_t* src, uint16_t* dst,
+                              void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if (!head_kind || !src || !dst || src == dst) return SVG_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return SVG_ERR_ALIGNMENT;
+  RowmapArgs a{};
+  a.g = make_geometry(s, nullptr);
+  a.flags = kRowmapInverse;
+  a.ntensor = 1;
+  a.norm_tensors = 0;
+  a.src[0] = src;
+  a.dst[0] = dst;
+  a.kind = head_kind;
+  return launch_rowmap(a, s->d, static_cast<cudaStream_t>(stream));
+}
+
+svg_status svg_profile_heads(const svg_shape* s, const svg_params* p, const uint16_t* qn, const uint16_t* kn,
+                             const uint16_t* v, const int32_t* sample_idx, int n, void* workspace,
+                             size_t workspace_bytes, float* mse_out, uint8_t* head_kind_out, void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if ((st = check_params(s, p, false)) != SVG_OK) return st;
+  if (!qn || !kn || !v || !sample_idx || !workspace || !head_kind_out) return SVG_ERR_INVALID_ARG;
+  if (n < 1 || n > kProfRows) return SVG_ERR_INVALID_ARG;
+  const void* ptrs[] = {qn, kn, v, workspace, mse_out};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return SVG_ERR_ALIGNMENT;
+  if (workspace_bytes < svg_profile_workspace_size(s, n)) return SVG_ERR_CAPACITY;
+  ProfArgs a{};
+  a.g = make_geometry(s, p);
+  a.scale_log2 = scale_of(s, p) * 1.4426950408889634f;
+  a.q = qn;
+  a.k = kn;
+  a.v = v;
+  a.sample = sample_idx;
+  a.n = n;
+  a.nchunk = prof_chunks(a.g.BH, a.g.L);
+  const int ntiles = (a.g.L + kProfKeys - 1) / kProfKeys;
+  a.tiles_per_chunk = (ntiles + a.nchunk - 1) / a.nchunk;
+  a.ws = static_cast<float*>(workspace);
+  a.mse_out = mse_out;
+  a.kind_out = head_kind_out;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  dim3 grid(a.nchunk, a.g.BH);
+  if (s->d == 128) {
+    if (!set_smem(profile_partial_kernel<128>, ProfSmem<128>::BYTES)) return SVG_ERR_CUDA;
+    profile_partial_kernel<128><<<grid, kProfThreads, ProfSmem<128>::BYTES, cs>>>(a);
+    if ((st = launch_status()) != SVG_OK) return st;
+    profile_combine_kernel<128><<<a.g.BH, 256, 0, cs>>>(a);
+  } else {
+    if (!set_smem(profile_partial_kernel<64>, ProfSmem<64>::BYTES)) return SVG_ERR_CUDA;
+    profile_partial_kernel<64><<<grid, kProfThreads, ProfSmem<64>::BYTES, cs>>>(a);
+    if ((st = launch_status()) != SVG_OK) return st;
+    profile_combine_kernel<64><<<a.g.BH, 256, 0, cs>>>(a);
+  }
+  return launch_status();
+}
+
+svg_status svg_build_block_index(const svg_shape* s, const svg_params* p, const uint8_t* head_kind,
+                                 int32_t* row_ptr, int32_t* col, uint8_t* full, int64_t capacity, void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if ((st = check_params(s, p, true)) != SVG_OK) return st;
+  if (!head_kind || !row_ptr || !col || !full || capacity < 0) return SVG_ERR_INVALID_ARG;
+  const Geometry g = make_geometry(s, p);
+  const int64_t n = static_cast<int64_t>(g.BH) * g.nqb;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  block_count_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, cs>>>(g, head_kind, row_ptr);
+  if ((st = launch_status()) != SVG_OK) return st;
+  block_scan_kernel<<<1, 1024, 0, cs>>>(row_ptr, n, capacity);
+  if ((st = launch_status()) != SVG_OK) return st;
+  block_fill_kernel<<<static_cast<unsigned>((n * 32 + 255) / 256), 256, 0, cs>>>(g, head_kind, row_ptr, col, full,
+                                                                                capacity);
+  return launch_status();
+}
+
+svg_status svg_block_sparse_attn(const svg_shape* s, const svg_params* p, const uint16_t* q, const uint16_t* k,
+                                 const uint16_t* v, const uint8_t* head_kind, const int32_t* row_ptr,
+                                 const int32_t* col, const uint8_t* full, uint16_t* out, float* lse_out,
+                                 void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if ((st = check_params(s, p, true)) != SVG_OK) return st;
+  if (!q || !k || !v || !head_kind || !row_ptr || !col || !full || !out) return SVG_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, out};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return SVG_ERR_ALIGNMENT;
+  if (out == q || out == k || out == v) return SVG_ERR_INVALID_ARG;
+  AttnArgs a{};
+  a.g = make_geometry(s, p);
+  a.scale_log2 = scale_of(s, p) * 1.4426950408889634f;
+  a.kind = head_kind;
+  a.row_ptr = row_ptr;
+  a.col = col;
+  a.full = full;
+  a.out = out;
+  a.lse = lse_out;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, s->d, s->L, a.g.BH, 128) || !make_map(&mk, k, s->d, s->L, a.g.BH, 64) ||
+      !make_map(&mv, v, s->d, s->L, a.g.BH, 64))
+    return SVG_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(a.g.BH) * static_cast<unsigned>(a.g.nqb);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (s->d == 128) {
+    if (!set_smem(attn_kernel<128>, AttnCfg<128>::SMEM_BYTES)) return SVG_ERR_CUDA;
+    attn_kernel<128><<<grid, AttnCfg<128>::THREADS, AttnCfg<128>::SMEM_BYTES, cs>>>(mq, mk, mv, a);
+  } else {
+    if (!set_smem(attn_kernel<64>, AttnCfg<64>::SMEM_BYTES)) return SVG_ERR_CUDA;
+    attn_kernel<64><<<grid, AttnCfg<64>::THREADS, AttnCfg<64>::SMEM_BYTES, cs>>>(mq, mk, mv, a);
+  }
+  return launch_status();
+}
+
+svg_status svg_attention_step(const svg_shape* s, const svg_params* p, const uint16_t* q, const uint16_t* k,
+                              const uint16_t* v, const float* gamma_q, const float* gamma_k, const float* rope_table,
+                              const int32_t* sample_idx, int n, const uint8_t* head_kind_in, uint16_t* qn,
+                              uint16_t* kn, uint16_t* qp, uint16_t* kp, uint16_t* vp, uint16_t* op, uint16_t* out,
+                              uint8_t* head_kind_out, float* mse_out, int32_t* row_ptr, int32_t* col, uint8_t* full,
+                              int64_t capacity, void* workspace, size_t workspace_bytes, void* stream) {
+  svg_status st;
+  if (!head_kind_out) return SVG_ERR_INVALID_ARG;
+  if ((st = svg_qknorm_rope_layout(s, p, SVG_NORM_ROPE, q, k, nullptr, gamma_q, gamma_k, rope_table, nullptr, qn, kn,
+                                   nullptr, stream)) != SVG_OK)
+    return st;
+  const uint8_t* kinds = head_kind_in;
+  if (!kinds) {
+    if ((st = svg_profile_heads(s, p, qn, kn, v, sample_idx, n, workspace, workspace_bytes, mse_out, head_kind_out,
+                                stream)) != SVG_OK)
+      return st;
+    kinds = head_kind_out;
+  }
+  if ((st = svg_build_block_index(s, p, kinds, row_ptr, col, full, capacity, stream)) != SVG_OK) return st;
+  if ((st = svg_qknorm_rope_layout(s, p, SVG_LAYOUT, qn, kn, v, nullptr, nullptr, nullptr, kinds, qp, kp, vp,
+                                   stream)) != SVG_OK)
+    return st;
+  if ((st = svg_block_sparse_attn(s, p, qp, kp, vp, kinds, row_ptr, col, full, op, nullptr, stream)) != SVG_OK)
+    return st;
+  return svg_inverse_layout(s, kinds, op, out, stream);
+}
+
+}  // extern "C"

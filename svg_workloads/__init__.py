@@ -213,19 +213,22 @@ def make_inputs(wl: Workload, seed: int | None = None, with_qkv: bool = True) ->
     return out
 
 
-def random_rows(wl: Workload, n_per_head: int, seed: int, boundary: bool = True) -> np.ndarray:
+def random_rows(wl: Workload, n_per_head: int, seed: int, boundary: bool = True,
+                max_boundary_tiles: int | None = None) -> np.ndarray:
     """Global row ids (b*H+h)*L + token for sampled checking: n random tokens per
-    head plus, if `boundary`, every token of each query tile that straddles a
-    frame boundary, the video/text boundary or the end of the sequence."""
+    head plus, if `boundary`, every token of query tiles that straddle a frame
+    boundary, the video/text boundary or the end of the sequence (at most
+    `max_boundary_tiles` of the frame-boundary tiles, chosen by the seed)."""
     rng = np.random.Generator(np.random.PCG64(seed))
     toks = set()
     if boundary:
-        cuts = {wl.Lv, wl.L - 1} | {f * wl.S for f in range(1, wl.F)}
-        for c in cuts:
+        frame_cuts = [f * wl.S for f in range(1, wl.F)]
+        if max_boundary_tiles is not None and len(frame_cuts) > max_boundary_tiles:
+            frame_cuts = sorted(rng.choice(frame_cuts, max_boundary_tiles, replace=False).tolist())
+        for c in list(frame_cuts) + [wl.Lv, wl.L - 1]:
             qb = min(c, wl.L - 1) // wl.bq
             toks.update(range(qb * wl.bq, min(wl.L, (qb + 1) * wl.bq)))
-        # the last tile (ragged tail)
-        toks.update(range((wl.nqb - 1) * wl.bq, wl.L))
+        toks.update(range((wl.nqb - 1) * wl.bq, wl.L))     # the ragged last tile
     toks = np.array(sorted(toks), np.int64)
     rows = []
     for bh in range(wl.B * wl.H):

@@ -1,0 +1,112 @@
+"""The C-ABI library loads, exports every declared symbol, and its host-side
+logic (argument checks, helpers) works without a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import svg_workloads as W
+from sparse_attention_video_qk_b200 import _lib as C
+from sparse_attention_video_qk_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return C.lib()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "svg.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(svg_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    syms = declared_symbols()
+    assert len(syms) >= 12
+    for s in syms:
+        assert hasattr(L, s), s
+    assert set(syms) == set(C.SIGNATURES), set(syms) ^ set(C.SIGNATURES)
+
+
+def test_version_and_status_strings(L):
+    assert b"sm_100a" in L.svg_version()
+    for st in range(8):
+        assert L.svg_status_string(st)
+
+
+def test_sample_queries_matches_generator(L):
+    for seed, Lv, n in [(1000, 256, 16), (1003, 118800, 64), (7, 10, 10), (5, 1 << 20, 64)]:
+        assert np.array_equal(api.sample_queries(seed, Lv, n), W.sample_queries(seed, Lv, n))
+    out = api.sample_queries(3, 50, 50)
+    assert sorted(out.tolist()) == list(range(50))          # n = Lv: a permutation
+    with pytest.raises(C.SVGError):
+        api.sample_queries(1, 10, 11)
+
+
+def test_rope_table_values(L):
+    wl = W.CONFIGS[0]
+    pb = api.Problem.from_workload(wl)
+    tab = api.rope_table(pb)
+    n0, n1, n2 = wl.rope_split
+    assert tab.size == 2 * (wl.F * n0 // 2 + wl.Hs * n1 // 2 + wl.Ws * n2 // 2)
+    cs = tab.reshape(-1, 2)
+    # position 0 rows are (1, 0); every entry lies on the unit circle
+    assert np.allclose(cs[: n0 // 2], [1.0, 0.0])
+    assert np.allclose((cs ** 2).sum(1), 1.0, atol=1e-6)
+    # frame 1, pair j: angle base^(-2j/n0)
+    j = np.arange(n0 // 2)
+    ang = np.arctan2(cs[n0 // 2: n0, 1], cs[n0 // 2: n0, 0])
+    assert np.allclose(ang, wl.rope_base ** (-2 * j / n0), atol=1e-6)
+
+
+def test_capacity_and_workspace(L):
+    wl = W.CONFIGS[3]
+    pb = api.Problem.from_workload(wl)
+    assert api.block_index_capacity(pb) == wl.H * wl.nqb * wl.nkb
+    ws = api.profile_workspace_size(pb, 64)
+    assert ws > 0 and ws % 16 == 0
+
+
+def _call_attn(L, sh, pr, ptr=16):
+    p = ctypes.c_void_p(ptr)
+    return L.svg_block_sparse_attn(ctypes.byref(sh), ctypes.byref(pr), p, p, p, p, p, p, p,
+                                   ctypes.c_void_p(ptr + 4096), None, None)
+
+
+def test_host_side_argument_errors(L):
+    """Errors are returned before anything touches the GPU."""
+    pb = api.Problem.from_workload(W.CONFIGS[0])
+    sh, pr = pb.c_shape(), pb.c_params()
+    bad = C.SvgShape(sh.B, sh.H, sh.L + 1, sh.d, sh.F, sh.Hs, sh.Ws, sh.text_len)
+    assert _call_attn(L, bad, pr) == C.SVG_ERR_SHAPE
+    d96 = C.SvgShape(sh.B, sh.H, sh.L, 96, sh.F, sh.Hs, sh.Ws, sh.text_len)
+    assert _call_attn(L, d96, pr) == C.SVG_ERR_UNSUPPORTED
+    pr32 = pb.c_params()
+    pr32.block_k = 32
+    assert _call_attn(L, sh, pr32) == C.SVG_ERR_UNSUPPORTED
+    assert _call_attn(L, sh, pr, ptr=8) == C.SVG_ERR_ALIGNMENT
+    neg = pb.c_params()
+    neg.spatial_frames = -1
+    assert _call_attn(L, sh, neg) == C.SVG_ERR_INVALID_ARG
+    p = ctypes.c_void_p(16)
+    # missing gamma with NORM_ROPE
+    assert L.svg_qknorm_rope_layout(ctypes.byref(sh), ctypes.byref(pr), C.SVG_NORM_ROPE, p, p, None, None, None,
+                                    None, None, ctypes.c_void_p(32), ctypes.c_void_p(48), None,
+                                    None) == C.SVG_ERR_INVALID_ARG
+    # bad rope split
+    prs = pb.c_params()
+    prs.rope_split[0] += 2
+    g = ctypes.c_void_p(64)
+    assert L.svg_qknorm_rope_layout(ctypes.byref(sh), ctypes.byref(prs), C.SVG_NORM_ROPE, p, p, None, g, g, g, None,
+                                    ctypes.c_void_p(32), ctypes.c_void_p(48), None, None) == C.SVG_ERR_SHAPE
+    # profiling: n out of range, workspace too small
+    assert L.svg_profile_heads(ctypes.byref(sh), ctypes.byref(pr), p, p, p, p, 65, p, 1 << 30, None, p,
+                               None) == C.SVG_ERR_INVALID_ARG
+    assert L.svg_profile_heads(ctypes.byref(sh), ctypes.byref(pr), p, p, p, p, 16, p, 16, None, p,
+                               None) == C.SVG_ERR_CAPACITY

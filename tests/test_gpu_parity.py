@@ -1,0 +1,295 @@
+"""Parity of every stage of the CUDA path with the fp64 oracle, through the C ABI.
+
+Bars (exactness where the stage is integer/bit work, the attention tolerance
+for floating point):
+  * QK-Norm + RoPE: within 1 bf16 ulp of the oracle's rounded fp64 result plus
+    2^-20 of the RoPE pair's norm (fp32 cancellation), >= 99% bit-equal;
+  * layout / inverse layout, block index lists, head choices: bit-exact;
+  * attention: max-abs <= 2e-2 and mean-abs <= 2e-3 against fp64, on the
+    oracle's own normalised inputs.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_attention_video_qk_b200 as svg
+import svg_workloads as W
+from gpu_util import assert_attention_close, assert_norm_rope_close, dev, f64, host_bits
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, MEAN_ABS = 2e-2, 2e-3
+
+
+@functools.lru_cache(maxsize=None)
+def case(key):
+    """Inputs and oracle stage-1 results of a named case (cached)."""
+    wl = CASES[key]
+    inp = W.make_inputs(wl)
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    qn = oracle.qknorm_rope(sh, pr, inp["q"], inp["gamma_q"])
+    kn = oracle.qknorm_rope(sh, pr, inp["k"], inp["gamma_k"])
+    return wl, inp, qn, kn
+
+
+CASES = {
+    "cfg0": W.CONFIGS[0],
+    "cfg1": W.CONFIGS[1],
+    "cfg2": W.CONFIGS[2],
+    "cfg3": W.CONFIGS[3],
+    # ragged: L = 116 is a multiple of neither tile size; text present; d = 128
+    "ragged128": W.small_workload(d=128, H=3, F=3, Hs=5, Ws=7, T=11, w=1, r=6, n_samples=12, bq=128),
+    # tiny: L = 11 < one tile
+    "tiny64": W.small_workload(d=64, H=2, F=1, Hs=2, Ws=3, T=5, w=0, r=1, n_samples=4, bq=64),
+    # several frames per key tile (S = 20), bq = 64
+    "smallS": W.small_workload(d=64, H=4, F=9, Hs=4, Ws=5, T=3, w=2, r=4, n_samples=16, bq=64),
+    # one frame: the temporal layout is the identity
+    "oneframe": W.small_workload(d=128, H=2, F=1, Hs=12, Ws=20, T=7, w=0, r=30, n_samples=8),
+    # wide windows that reduce to dense
+    "wide": W.small_workload(d=64, H=2, F=5, Hs=6, Ws=7, T=9, w=4, r=41, n_samples=8),
+}
+FULL_ROW_CASES = ("cfg0", "ragged128", "tiny64", "smallS", "oneframe", "wide")
+
+
+def pb_of(wl):
+    return svg.Problem.from_workload(wl)
+
+
+def mixed_kinds(H):
+    return np.array([(W.SPATIAL, W.TEMPORAL, W.DENSE)[h % 3] for h in range(H)], np.uint8)
+
+
+def rows_for(key, wl):
+    if key in FULL_ROW_CASES:
+        return np.arange(wl.B * wl.H * wl.L, dtype=np.int64)
+    if key == "cfg3":
+        return W.random_rows(wl, 48, seed=11, max_boundary_tiles=1)
+    return W.random_rows(wl, 96, seed=11, max_boundary_tiles=3)
+
+
+# ------------------------------------------------------------ QK-Norm + RoPE
+
+@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "ragged128", "tiny64", "oneframe"])
+def test_qknorm_rope_within_one_ulp(key):
+    wl, inp, qn_ref, kn_ref = case(key)
+    pb = pb_of(wl)
+    table = dev(svg.rope_table(pb))
+    qn, kn = svg.qknorm_rope(pb, dev(inp["q"]), dev(inp["k"]), dev(inp["gamma_q"]), dev(inp["gamma_k"]), table)
+    svg.sync_status()
+    for got, ref, name in ((host_bits(qn), qn_ref, "q"), (host_bits(kn), kn_ref, "k")):
+        assert_norm_rope_close(got, ref, f"{key}/{name}")
+
+
+def test_qknorm_rope_cfg3_sampled_rows():
+    wl = W.CONFIGS[3]
+    inp = W.make_inputs(wl)
+    pb = pb_of(wl)
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    rows = W.random_rows(wl, 256, seed=5, max_boundary_tiles=2)
+    qn, kn = svg.qknorm_rope(pb, dev(inp["q"]), dev(inp["k"]), dev(inp["gamma_q"]), dev(inp["gamma_k"]),
+                             dev(svg.rope_table(pb)))
+    svg.sync_status()
+    for got_t, x, gname in ((qn, inp["q"], "gamma_q"), (kn, inp["k"], "gamma_k")):
+        got = host_bits(got_t).reshape(-1, wl.d)[rows]
+        ref = oracle.f64_to_bf16(oracle.qknorm_rope_f64(sh, pr, x, inp[gname], rows))
+        assert_norm_rope_close(got, ref, gname)
+
+
+# ------------------------------------------------------------------ layout
+
+@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "ragged128", "tiny64", "smallS", "oneframe"])
+def test_layout_and_inverse_bit_exact(key):
+    wl, inp, _, _ = case(key)
+    pb = pb_of(wl)
+    sh = oracle.shape_of(wl)
+    kinds = mixed_kinds(wl.H)
+    q, k, v = dev(inp["q"]), dev(inp["k"]), dev(inp["v"])
+    qp, kp, vp = svg.layout(pb, q, k, v, dev(kinds))
+    back = svg.inverse_layout(pb, dev(kinds), qp)
+    svg.sync_status()
+    for got, name in ((qp, "q"), (kp, "k"), (vp, "v")):
+        assert np.array_equal(host_bits(got), oracle.layout(sh, kinds, inp[name])), name
+    assert np.array_equal(host_bits(back), inp["q"])
+    assert np.array_equal(host_bits(svg.inverse_layout(pb, dev(kinds), vp)),
+                          oracle.layout(sh, kinds, oracle.layout(sh, kinds, inp["v"]), inverse=True))
+
+
+@pytest.mark.parametrize("key", ["cfg0", "ragged128", "smallS"])
+def test_fused_norm_rope_layout(key):
+    """flags = NORM_ROPE | LAYOUT equals the two separate passes bit for bit."""
+    wl, inp, _, _ = case(key)
+    pb = pb_of(wl)
+    kinds = dev(mixed_kinds(wl.H))
+    args = (dev(inp["q"]), dev(inp["k"]))
+    g = (dev(inp["gamma_q"]), dev(inp["gamma_k"]), dev(svg.rope_table(pb)))
+    qn, kn = svg.qknorm_rope(pb, *args, *g)
+    two = svg.layout(pb, qn, kn, dev(inp["v"]), kinds)
+    one = svg.qknorm_rope_layout(pb, *args, dev(inp["v"]), *g, kinds, flags=3)
+    svg.sync_status()
+    for a, b in zip(one, two):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+# ------------------------------------------------------------- block index
+
+def csr_host(row_ptr, col, full):
+    rp = row_ptr.cpu().numpy()
+    nnz = int(rp[-1])
+    return rp, col[:nnz].cpu().numpy(), full[:nnz].cpu().numpy()
+
+
+@pytest.mark.parametrize("key,kinds_mode", [("cfg0", "mixed"), ("cfg1", "mixed"), ("cfg2", "mixed"),
+                                            ("ragged128", "mixed"), ("tiny64", "mixed"), ("smallS", "mixed"),
+                                            ("oneframe", "mixed"), ("wide", "mixed"), ("cfg3", "planted")])
+def test_block_index_bit_exact(key, kinds_mode):
+    wl = CASES[key]
+    pb = pb_of(wl)
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    kinds = mixed_kinds(wl.H) if kinds_mode == "mixed" else \
+        np.array([W.SPATIAL if c == "S" else W.TEMPORAL for c in wl.planted], np.uint8)
+    rp, col, full = csr_host(*svg.build_block_index(pb, dev(kinds)))
+    svg.sync_status()
+    rp_ref, col_ref, full_ref = oracle.block_list(sh, pr, kinds)
+    assert np.array_equal(rp, rp_ref)
+    assert np.array_equal(col, col_ref)
+    assert np.array_equal(full, full_ref)
+
+
+def test_block_index_capacity_overflow_is_reported():
+    wl = CASES["smallS"]
+    pb = pb_of(wl)
+    kinds = dev(np.full(wl.H, W.DENSE, np.uint8))
+    need = wl.H * wl.nqb * wl.nkb
+    cap = need // 2
+    col = torch.full((need,), -7, dtype=torch.int32, device="cuda")
+    full = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    row_ptr = torch.empty(wl.H * wl.nqb + 1, dtype=torch.int32, device="cuda")
+    svg.build_block_index(pb, kinds, capacity=cap, out=(row_ptr, col, full))
+    with pytest.raises(svg.SVGError) as e:
+        svg.sync_status()
+    assert e.value.status == 5
+    assert (col[cap:].cpu().numpy() == -7).all()          # nothing written past capacity
+    svg.sync_status()                                     # the error word was cleared
+
+
+# --------------------------------------------------------------- profiling
+
+@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "smallS", "ragged128", "cfg3"])
+def test_profile_choices_bit_exact(key):
+    wl, inp, qn, kn = case(key)
+    pb = pb_of(wl)
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    mse_ref, kinds_ref = oracle.profile(sh, pr, qn, kn, inp["v"], inp["sample_idx"])
+    kinds, mse = svg.profile_heads(pb, dev(qn), dev(kn), dev(inp["v"]), dev(inp["sample_idx"]))
+    svg.sync_status()
+    kinds = kinds.cpu().numpy()
+    mse = mse.cpu().numpy().astype(np.float64)
+    gap = np.abs(mse_ref[:, 0] - mse_ref[:, 1]) / mse_ref.max(1)
+    near_tie = gap < 1e-4
+    assert np.array_equal(kinds[~near_tie], kinds_ref[~near_tie]), (kinds, kinds_ref, gap)
+    assert near_tie.sum() == 0, f"near-ties: {np.nonzero(near_tie)[0]}"
+    rel = np.abs(mse - mse_ref) / mse_ref
+    assert rel.max() < 2e-2, rel.max()
+    planted = inp["planted"]
+    if key in ("cfg0", "cfg2", "cfg3"):
+        sel = planted != 255
+        assert np.array_equal(kinds[sel], planted[sel])
+
+
+def test_profile_bad_sample_index_reported():
+    wl, inp, qn, kn = case("cfg0")
+    pb = pb_of(wl)
+    bad = inp["sample_idx"].copy()
+    bad[3] = wl.L + 5
+    svg.profile_heads(pb, dev(qn), dev(kn), dev(inp["v"]), dev(bad))
+    with pytest.raises(svg.SVGError) as e:
+        svg.sync_status()
+    assert e.value.status == 1
+
+
+# --------------------------------------------------------------- attention
+
+def run_sparse(wl, qn, kn, v, kinds, want_lse=False):
+    pb = pb_of(wl)
+    kd = dev(kinds)
+    qp, kp, vp = svg.layout(pb, dev(qn), dev(kn), dev(v), kd)
+    row_ptr, col, full = svg.build_block_index(pb, kd)
+    res = svg.block_sparse_attn(pb, qp, kp, vp, kd, row_ptr, col, full, want_lse=want_lse)
+    op, lse = res if want_lse else (res, None)
+    out = svg.inverse_layout(pb, kd, op)
+    svg.sync_status()
+    return out, lse
+
+
+@pytest.mark.parametrize("key", ["cfg0", "ragged128", "tiny64", "smallS", "oneframe", "wide", "cfg1", "cfg2"])
+@pytest.mark.parametrize("kinds_mode", ["mixed", "spatial", "temporal"])
+def test_attention_parity(key, kinds_mode):
+    wl, inp, qn, kn = case(key)
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    kinds = {"mixed": mixed_kinds(wl.H), "spatial": np.zeros(wl.H, np.uint8),
+             "temporal": np.ones(wl.H, np.uint8)}[kinds_mode]
+    out, lse = run_sparse(wl, qn, kn, inp["v"], kinds, want_lse=True)
+    rows = rows_for(key, wl)
+    ref, ref_lse = oracle.attention_rows(sh, pr, kinds, qn, kn, inp["v"], rows, want_lse=True)
+    got = host_bits(out).reshape(-1, wl.d)[rows]
+    assert_attention_close(got, ref, MAX_ABS, MEAN_ABS, f"{key}/{kinds_mode}")
+    # LSE is stored in the head's layout order
+    lse_h = lse.cpu().numpy().reshape(wl.B * wl.H, wl.L)
+    bh, tok = rows // wl.L, rows % wl.L
+    pos = np.array([oracle.perm(sh, int(kinds[b]), int(t)) for b, t in zip(bh, tok)])
+    assert np.abs(lse_h[bh, pos] - ref_lse).max() < 5e-3
+
+
+def test_attention_dense_kinds_equal_dense_attention():
+    wl, inp, qn, kn = case("smallS")
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    kinds = np.full(wl.H, W.DENSE, np.uint8)
+    out, _ = run_sparse(wl, qn, kn, inp["v"], kinds)
+    rows = np.arange(wl.H * wl.L, dtype=np.int64)
+    ref = oracle.attention_rows(sh, pr, kinds, qn, kn, inp["v"], rows)
+    assert_attention_close(host_bits(out).reshape(-1, wl.d), ref, MAX_ABS, MEAN_ABS, "dense")
+
+
+def test_attention_cfg3_sampled_rows():
+    wl, inp, qn, kn = case("cfg3")
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    kinds = np.array([W.SPATIAL if c == "S" else W.TEMPORAL for c in wl.planted], np.uint8)
+    out, _ = run_sparse(wl, qn, kn, inp["v"], kinds)
+    rows = rows_for("cfg3", wl)
+    ref = oracle.attention_rows(sh, pr, kinds, qn, kn, inp["v"], rows)
+    assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, "cfg3")
+
+
+# ---------------------------------------------------------------- full step
+
+@pytest.mark.parametrize("key", ["cfg0", "smallS", "cfg1", "cfg2"])
+def test_full_step_end_to_end(key):
+    wl, inp, qn, kn = case(key)
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    pb = pb_of(wl)
+    buf = svg.StepBuffers(pb, wl.n_samples)
+    out = svg.attention_step(pb, dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["gamma_q"]),
+                             dev(inp["gamma_k"]), dev(inp["sample_idx"]), buf)
+    svg.sync_status()
+    _, kinds_ref = oracle.profile(sh, pr, qn, kn, inp["v"], inp["sample_idx"])
+    assert np.array_equal(buf.kinds.cpu().numpy(), kinds_ref)
+    rows = rows_for(key, wl)
+    ref = oracle.attention_rows(sh, pr, kinds_ref, qn, kn, inp["v"], rows)
+    assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, key)
+
+
+def test_host_buffer_api_matches_device_api():
+    wl, inp, _, _ = case("cfg0")
+    pb = pb_of(wl)
+    pin = lambda a: torch.from_numpy(a).view(torch.bfloat16).pin_memory()
+    out_h = svg.sparse_attention(pb, pin(inp["q"]), pin(inp["k"]), pin(inp["v"]), torch.from_numpy(inp["gamma_q"]),
+                                 torch.from_numpy(inp["gamma_k"]), torch.from_numpy(inp["sample_idx"]))
+    torch.cuda.synchronize()
+    buf = svg.StepBuffers(pb, wl.n_samples)
+    out_d = svg.attention_step(pb, dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["gamma_q"]),
+                               dev(inp["gamma_k"]), dev(inp["sample_idx"]), buf)
+    svg.sync_status()
+    assert torch.equal(out_h.view(torch.int16), out_d.cpu().view(torch.int16))
