@@ -77,28 +77,37 @@ def traffic_from_profile(kernel_file: str, summary: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """nvidia-smi clock / throttle sampling; only samples whose timestamp falls
+    inside [window start, window end] (host clock) are summarised."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.t0 = self.t1 = None
+        self.out = ""
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
-        time.sleep(0.3)
+        time.sleep(0.5)
         return self
 
+    def start(self):
+        self.t0 = time.time()
+
+    def stop(self):
+        self.t1 = time.time()
+
     def __exit__(self, *a):
-        self.out = ""
+        time.sleep(0.2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -108,24 +117,33 @@ class ClockSampler:
                 self.out, _ = self.proc.communicate()
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        from datetime import datetime
+        sm, mx, reasons, power = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in (self.out or "").strip().splitlines():
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                ts = datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                clk, mxc = float(f[1]), float(f[2])
             except ValueError:
                 continue
+            if self.t0 is not None and not (self.t0 <= ts <= self.t1):
+                continue
+            sm.append(clk)
+            mx = mxc
+            try:
+                power.append(float(f[3]))
+            except ValueError:
+                pass
             for n, v in zip(names, f[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "power_w_median": statistics.median(power) if power else None}
 
 
 # ---------------------------------------------------------------- GPU arm --
@@ -144,7 +162,6 @@ def run_gpu(args, rank, world, local_rank):
     pin = lambda a, bf=True: (torch.from_numpy(a).view(torch.bfloat16) if bf else torch.from_numpy(a)).pin_memory()
     q_h, k_h, v_h = pin(inp["q"]), pin(inp["k"]), pin(inp["v"])
     gq_h, gk_h, si_h = pin(inp["gamma_q"], False), pin(inp["gamma_k"], False), pin(inp["sample_idx"], False)
-    del inp
     q, k, v = (t.to(device) for t in (q_h, k_h, v_h))
     gq, gk, si = gq_h.to(device), gk_h.to(device), si_h.to(device)
     buf = svg.StepBuffers(pb, int(si.numel()), device)
@@ -199,12 +216,14 @@ def run_gpu(args, rank, world, local_rank):
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
+        clk.start()
         t_start.record(stream)
         for s in range(args.steps):
             ev[s][0].record(stream)
             one_step(ev[s])
         t_end.record(stream)
         torch.cuda.synchronize()
+        clk.stop()
     if world > 1:
         dist.barrier()
     svg.sync_status()
@@ -316,19 +335,18 @@ def run_gpu(args, rank, world, local_rank):
         "clocks": clocks,
     }
     if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_rows)
+        line["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_rows)
     return line
 
 
 # ---------------------------------------------------------- oracle (CPU) --
 
-def oracle_sample_rate(wl, n_rows: int, seed: int = 0):
+def oracle_sample_rate(wl, inp, n_rows: int, seed: int = 0):
     """Times the fp64 oracle on a bounded sample of the step: QK-Norm+RoPE of
     the sampled rows' Q and of K, and masked attention of `n_rows` query rows
     spread over the heads (planted head kinds).  Returns (TFLOP/s counted like
     the GPU metric, seconds, threads, description)."""
     import oracle
-    inp = W.make_inputs(wl)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
     kinds = np.array([0 if c == "S" else 1 for c in wl.planted], np.uint8)
     rng = np.random.Generator(np.random.PCG64(seed))
@@ -381,8 +399,8 @@ def kept_cols_closed(wl, kind, qb):
     return int(sum(min(bk, L - kb * bk) for kb in kbs))
 
 
-def cpu_baseline(wl, n_rows):
-    rate, secs, threads, desc = oracle_sample_rate(wl, n_rows)
+def cpu_baseline(wl, inp, n_rows):
+    rate, secs, threads, desc = oracle_sample_rate(wl, inp, n_rows)
     return {"value": round(rate, 8), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": desc, "seconds": round(secs, 2)}
 
@@ -391,9 +409,10 @@ def run_reference(args, rank):
     if rank != 0:
         return None
     wl = W.CONFIGS[args.config]
+    inp = W.make_inputs(wl)
     rates, secs_all = [], []
     for s in range(args.warmup + args.steps):
-        rate, secs, threads, desc = oracle_sample_rate(wl, args.ref_rows, seed=s)
+        rate, secs, threads, desc = oracle_sample_rate(wl, inp, args.ref_rows, seed=s)
         if s >= args.warmup:
             rates.append(rate)
             secs_all.append(secs)
@@ -417,12 +436,12 @@ def run_reference(args, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--config", type=int, default=3)
-    ap.add_argument("--cpu-rows", type=int, default=480)
-    ap.add_argument("--ref-rows", type=int, default=240)
+    ap.add_argument("--cpu-rows", type=int, default=1920)
+    ap.add_argument("--ref-rows", type=int, default=960)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
