@@ -118,6 +118,35 @@ svg_status svg_profile_heads(const svg_shape* shape, const svg_params* params,
                              const int32_t* sample_idx, int n, void* workspace, size_t workspace_bytes,
                              float* mse_out, uint8_t* head_kind_out, void* stream);
 
+/* Stage 2 without a caller-provided workspace.  The paper has no counterpart:
+ * this entry point exists for callers that can hand the library only their
+ * inputs and outputs and cannot allocate device memory themselves -- for
+ * example a plugin running inside a host runtime that owns all device memory
+ * and exposes no allocator, or a serving process that reserved its whole
+ * memory pool at start-up and must not call cudaMalloc while serving.
+ * It computes exactly what svg_profile_heads computes (same arguments minus
+ * the workspace) and allocates nothing: its scratch is a fixed 16 MiB device
+ * array inside the library, which every GPU that loads the library holds until
+ * the process exits.
+ *   - Size limit: one key chunk of partial results takes B*H*64*(4+3d)*4 bytes;
+ *     if that exceeds 16 MiB (B*H > 168 at d=128, > 334 at d=64) the call
+ *     returns SVG_ERR_CAPACITY and launches nothing.  Otherwise it splits the
+ *     keys into as many chunks as fit (at most as many as svg_profile_heads).
+ *   - Set-up: the first call on each device looks up the scratch's device
+ *     address (cudaGetSymbolAddress, with that device current) and caches it;
+ *     make that first call before any stream capture.
+ *   - Sharing: every call uses the same scratch and leaves its contents behind.
+ *     Each call writes every scratch entry it later reads, so nothing needs to
+ *     start at zero; but two calls whose kernels overlap on the GPU (different
+ *     streams, or different host threads) race on the scratch and corrupt each
+ *     other's results.  Serialise them.
+ * Errors are reported as for svg_profile_heads (SVG_ERR_CUDA if the set-up
+ * lookup fails). */
+svg_status svg_profile_heads_noalloc(const svg_shape* shape, const svg_params* params,
+                                     const uint16_t* qn, const uint16_t* kn, const uint16_t* v,
+                                     const int32_t* sample_idx, int n,
+                                     float* mse_out, uint8_t* head_kind_out, void* stream);
+
 /* Block index (not on the pages; the block-sparse kernel they describe needs it).
  * In each head's layout, the tile (q-block qb: rows [qb*block_q, +block_q),
  * k-block kb: keys [kb*block_k, +block_k), rows/keys >= L excluded) is listed iff at

@@ -40,6 +40,7 @@ _SP, _PP = ctypes.POINTER(SvgShape), ctypes.POINTER(SvgParams)
 SIGNATURES = {
     "svg_qknorm_rope_layout": (_i32, [_SP, _PP, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "svg_profile_heads": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp, _vp, _vp]),
+    "svg_profile_heads_noalloc": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp]),
     "svg_build_block_index": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _i64, _vp]),
     "svg_block_sparse_attn": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "svg_inverse_layout": (_i32, [_SP, _vp, _vp, _vp, _vp]),

@@ -163,6 +163,21 @@ def profile_heads(pb: Problem, qn, kn, v, sample_idx, workspace=None, kinds_out=
     return kinds_out, mse_out
 
 
+def profile_heads_noalloc(pb: Problem, qn, kn, v, sample_idx, kinds_out=None, mse_out=None, stream=None):
+    """svg_profile_heads_noalloc: profiling with the library's fixed scratch
+    (no workspace argument).  Returns (kinds uint8 [B*H], mse fp32 [B*H, 2])."""
+    sh, pr = pb.c_shape(), pb.c_params()
+    n = int(sample_idx.numel())
+    if kinds_out is None:
+        kinds_out = torch.empty(pb.B * pb.H, dtype=torch.uint8, device=qn.device)
+    if mse_out is None:
+        mse_out = torch.empty(pb.B * pb.H, 2, dtype=torch.float32, device=qn.device)
+    st = lib().svg_profile_heads_noalloc(ctypes.byref(sh), ctypes.byref(pr), _p(qn), _p(kn), _p(v), _p(sample_idx),
+                                         n, _p(mse_out), _p(kinds_out), _stream(stream))
+    check(st, "svg_profile_heads_noalloc")
+    return kinds_out, mse_out
+
+
 def build_block_index(pb: Problem, kinds, capacity=None, out=None, stream=None):
     """Returns (row_ptr int32 [B*H*nqb+1], col int32 [capacity], full uint8 [capacity]).
     Only the first row_ptr[-1] entries of col/full are meaningful."""

@@ -437,3 +437,6 @@ svg_status svg_attention_step(const svg_shape* s, const svg_params* p, const uin
 }
 
 }  // extern "C"
+
+// Profiling with library-owned scratch (svg_profile_heads_noalloc).
+#include "profile_noalloc.cuh"
