@@ -6,9 +6,11 @@
 // layout transform, reaches close to the 1/density speedup.  This is a
 // B200-native design of that kernel:
 //
-//   * one CTA per (b, h, query tile of 128 rows); 6 warps:
-//       warp 0  TMA producer: Q once, then K and V tiles of the listed key
-//               blocks into an NS-stage shared-memory ring (128-byte swizzle);
+//   * one CTA per (b, h, query tile of 128 rows), text-row tiles first, then
+//     head by head for L2 reuse of each head's K and V; 6 warps:
+//       warp 0  TMA producer: Q once, then the K and V tiles of the listed
+//               key blocks into one ring of shared-memory slots (128-byte
+//               swizzle), K released after Q.K^T and V after P.V;
 //       warp 1  TMEM allocator and the single MMA-issuing thread;
 //       warps 2-5  softmax: thread = query row = TMEM lane.
 //   * two listed 64-key blocks (consecutive entries of the CSR list, not
@@ -42,13 +44,17 @@ struct AttnCfg {
   static constexpr int PANEL_Q = BM * 128;       // bytes of one Q panel
   static constexpr int PANEL_KV = BN * 128;      // bytes of one K / V panel
   static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;    // one K (or V) stage
-  static constexpr int NS = (D == 128) ? 2 : 4;  // pipeline stages
-  static constexpr int DATA_BYTES = Q_BYTES + 2 * NS * KV_BYTES;
-  static constexpr int SMEM_BYTES = DATA_BYTES + 256 + 1024;  // barriers + alignment slack
+  static constexpr int SLOT_BYTES = BN * D * 2;  // one K or one V tile
+  // K and V tiles share one ring of slots, filled in the order K0 V0 K1 V1 ...
+  static constexpr int NSLOT = (D == 128) ? 6 : 12;
+  static constexpr int DATA_BYTES = Q_BYTES + NSLOT * SLOT_BYTES;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMEM_BYTES = DATA_BYTES + BAR_BYTES + 1024;  // + alignment slack
   static constexpr int THREADS = 192;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(1 + 2 * NSLOT + 6 + 2 <= BAR_BYTES / 8, "barrier area");
 };
 
 struct AttnArgs {
@@ -69,6 +75,67 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (Blackwell f32x2 ALU ops): one instruction for two lanes of work.
+__device__ __forceinline__ uint64_t f32x2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on the FMA pipe for a pair (x <= 8): x = n + f with n = round(x) and
+// f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients
+// minimise the maximum relative error on that interval (Remez exchange, see
+// gen_exp2_poly.py; max relative error 7.5e-5, far below bf16's 2^-8); 2^n
+// is added to the exponent field.  The rounding uses the 1.5 * 2^23 shift:
+// the integer n lands in the low mantissa bits of t, and (bits(t) << 23) is
+// n << 23.  x is clamped at -125 so the result stays a normal float
+// (2^-125 ~ 2.4e-38 stands in for 0 on masked keys).
+#ifndef SVG_POLY_EVERY
+#define SVG_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = SVG_POLY_EVERY;   // every kPolyEvery-th pair uses the polynomial (0: never)
+constexpr int kPolyStride = kPolyEvery > 0 ? kPolyEvery : 1;
+
+__device__ __forceinline__ void poly_exp2x2(float x0, float x1, float& p0, float& p1) {
+  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
+  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
+  constexpr float c2 = 0.2426111251115799f, c3 = 0.0551716685295105f;
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  const uint64_t x = f32x2(x0, x1);
+  const uint64_t t = fadd2(x, f32x2(kShift, kShift));
+  uint64_t n;
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(n) : "l"(t), "l"(f32x2(kShift, kShift)));
+  uint64_t f;
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(f) : "l"(x), "l"(n));
+  uint64_t q = ffma2(f32x2(c3, c3), f, f32x2(c2, c2));
+  q = ffma2(q, f, f32x2(c1, c1));
+  q = ffma2(q, f, f32x2(c0, c0));
+  float q0, q1, t0, t1;
+  unpack2(q, q0, q1);
+  unpack2(t, t0, t1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
@@ -82,33 +149,47 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, const AttnArgs a) {
   using C = AttnCfg<D>;
-  constexpr int NS = C::NS;
+  constexpr int NSLOT = C::NSLOT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + C::Q_BYTES;
-  uint8_t* sV = sK + NS * C::KV_BYTES;
+  uint8_t* sKV = smem + C::Q_BYTES;              // NSLOT slots of SLOT_BYTES
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::DATA_BYTES);
   // barrier slots
   const uint32_t b_q = smem_addr(&bars[0]);
   auto b_full = [&](int s) { return smem_addr(&bars[1 + s]); };
-  auto b_empty = [&](int s) { return smem_addr(&bars[1 + NS + s]); };
-  auto b_s = [&](int b) { return smem_addr(&bars[1 + 2 * NS + b]); };
-  auto b_p = [&](int b) { return smem_addr(&bars[3 + 2 * NS + b]); };
-  const uint32_t b_o = smem_addr(&bars[5 + 2 * NS]);
-  const uint32_t b_drain = smem_addr(&bars[6 + 2 * NS]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[16]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[17]);
+  auto b_empty = [&](int s) { return smem_addr(&bars[1 + NSLOT + s]); };
+  auto b_s = [&](int b) { return smem_addr(&bars[1 + 2 * NSLOT + b]); };
+  auto b_p = [&](int b) { return smem_addr(&bars[3 + 2 * NSLOT + b]); };
+  const uint32_t b_o = smem_addr(&bars[5 + 2 * NSLOT]);
+  const uint32_t b_drain = smem_addr(&bars[6 + 2 * NSLOT]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[7 + 2 * NSLOT]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[8 + 2 * NSLOT]);
 
   const Geometry& g = a.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x % g.BH;
-  const int qb = g.nqb - 1 - static_cast<int>(blockIdx.x / g.BH);   // text-heavy tiles first
+  // Work order: first the query tiles that contain text rows (they attend to
+  // every key: the longest lists), then the rest head by head, so the CTAs
+  // resident at one time read the same head's keys and values out of L2.
+  int bh, qb;
+  {
+    const int qb_text = (g.T > 0) ? g.Lv / g.bq : g.nqb;   // first tile holding a text row
+    const int n_heavy = g.nqb - qb_text;
+    const int x = blockIdx.x;
+    if (x < g.BH * n_heavy) {
+      bh = x / n_heavy;
+      qb = qb_text + x % n_heavy;
+    } else {
+      const int y = x - g.BH * n_heavy;
+      bh = y / qb_text;
+      qb = y % qb_text;
+    }
+  }
   const int q_row0 = qb * g.bq;
 
   if (threadIdx.x == 0) {
     mbar_init(b_q, 1);
-    for (int s = 0; s < NS; s++) {
+    for (int s = 0; s < NSLOT; s++) {
       mbar_init(b_full(s), 1);
       mbar_init(b_empty(s), 1);
     }
@@ -134,6 +215,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Slot sequence i = 0, 1, 2, ...: K of tile i/2 for even i, V for odd i.
     if (lane == 0) {
       tma_prefetch_desc(&tmq);
       tma_prefetch_desc(&tmk);
@@ -141,31 +223,29 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       mbar_expect_tx(b_q, C::Q_BYTES);
 #pragma unroll
       for (int p = 0; p < C::PANELS; p++) tma_load_3d(smem_addr(sQ + p * C::PANEL_Q), &tmq, p * 64, q_row0, bh, b_q);
-      int issued[NS];
-#pragma unroll
-      for (int s = 0; s < NS; s++) issued[s] = 0;
-      for (int j = 0; j < nT; j++) {
-        const int st = j % NS;
-        if (j >= NS && !mbar_wait(b_empty(st), ((j / NS) - 1) & 1, abort_flag)) break;
-        const int e0 = rp0 + 2 * j;
+      int issued = 0;
+      for (int i = 0; i < 2 * nT; i++) {
+        const int st = i % NSLOT;
+        if (i >= NSLOT && !mbar_wait(b_empty(st), ((i / NSLOT) - 1) & 1, abort_flag)) break;
+        const int e0 = rp0 + 2 * (i >> 1);
         const int nb = min(2, rp1 - e0);
-        mbar_expect_tx(b_full(st), nb * 64 * D * 2 * 2);
+        const CUtensorMap* map = (i & 1) ? &tmv : &tmk;
+        mbar_expect_tx(b_full(st), nb * 64 * D * 2);
         for (int h = 0; h < nb; h++) {
           const int kb = a.col[e0 + h];
 #pragma unroll
           for (int p = 0; p < C::PANELS; p++) {
-            const uint32_t off = st * C::KV_BYTES + p * C::PANEL_KV + h * 64 * 128;
-            tma_load_3d(smem_addr(sK + off), &tmk, p * 64, kb * 64, bh, b_full(st));
-            tma_load_3d(smem_addr(sV + off), &tmv, p * 64, kb * 64, bh, b_full(st));
+            const uint32_t off = st * C::SLOT_BYTES + p * C::PANEL_KV + h * 64 * 128;
+            tma_load_3d(smem_addr(sKV + off), map, p * 64, kb * 64, bh, b_full(st));
           }
         }
-        issued[st]++;
+        issued = i + 1;
       }
       if (*abort_flag) {
         // let every issued copy land before the CTA exits
         mbar_wait_drain(b_q, 0);
-        for (int s = 0; s < NS; s++)
-          if (issued[s] > 0) mbar_wait_drain(b_full(s), (issued[s] - 1) & 1);
+        for (int i = max(0, issued - NSLOT); i < issued; i++)
+          mbar_wait_drain(b_full(i % NSLOT), (i / NSLOT) & 1);
       }
     }
   } else if (warp == 1) {
@@ -174,13 +254,14 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       constexpr uint32_t idS128 = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idS64 = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_base = smem_addr(sQ), k_base = smem_addr(sK), v_base = smem_addr(sV);
+      const uint32_t q_base = smem_addr(sQ), kv_base = smem_addr(sKV);
       bool ok = mbar_wait(b_q, 0, abort_flag);
       bool issued_any = false;
       for (int j = 0; ok && j <= nT; j++) {
         if (j < nT) {
-          const int st = j % NS;
-          if (!mbar_wait(b_full(st), (j / NS) & 1, abort_flag)) break;
+          // S_j = Q K_j^T; the K slot is released as soon as these MMAs finish
+          const int i = 2 * j, st = i % NSLOT;
+          if (!mbar_wait(b_full(st), (i / NSLOT) & 1, abort_flag)) break;
           tc_fence_after();
           const int nb = min(2, rp1 - (rp0 + 2 * j));
           const uint32_t dS = tmem + ((j & 1) ? C::TM_S1 : C::TM_S0);
@@ -189,22 +270,25 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             const uint32_t koff = (kk >> 2) * C::PANEL_KV + (kk & 3) * 32;
             const uint32_t qoff = (kk >> 2) * C::PANEL_Q + (kk & 3) * 32;
             const uint64_t da = sdesc_sw128(q_base + qoff, 16, 1024);
-            const uint64_t db = sdesc_sw128(k_base + st * C::KV_BYTES + koff, 16, 1024);
+            const uint64_t db = sdesc_sw128(kv_base + st * C::SLOT_BYTES + koff, 16, 1024);
             umma_ss(dS, da, db, nb == 2 ? idS128 : idS64, kk > 0);
           }
           umma_commit(b_s(j & 1));
+          umma_commit(b_empty(st));
           issued_any = true;
         }
         if (j >= 1) {
-          const int i = j - 1;
-          const int st = i % NS;
-          if (!mbar_wait(b_p(i & 1), (i >> 1) & 1, abort_flag)) break;
+          // O += P_{j-1} V_{j-1}
+          const int t = j - 1;
+          const int i = 2 * t + 1, st = i % NSLOT;
+          if (!mbar_wait(b_p(t & 1), (t >> 1) & 1, abort_flag)) break;
+          if (!mbar_wait(b_full(st), (i / NSLOT) & 1, abort_flag)) break;
           tc_fence_after();
-          const int nb = min(2, rp1 - (rp0 + 2 * i));
-          const uint32_t aP = tmem + ((i & 1) ? C::TM_S1 : C::TM_S0);
+          const int nb = min(2, rp1 - (rp0 + 2 * t));
+          const uint32_t aP = tmem + ((t & 1) ? C::TM_S1 : C::TM_S0);
           for (int kk = 0; kk < nb * 4; kk++) {
-            const uint64_t db = sdesc_sw128(v_base + st * C::KV_BYTES + kk * 2048, C::PANEL_KV, 1024);
-            umma_ts(tmem + C::TM_O, aP + kk * 8, db, idO, (i > 0 || kk > 0) ? 1u : 0u);
+            const uint64_t db = sdesc_sw128(kv_base + st * C::SLOT_BYTES + kk * 2048, C::PANEL_KV, 1024);
+            umma_ts(tmem + C::TM_O, aP + kk * 8, db, idO, (t > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(b_empty(st));
           umma_commit(b_o);
@@ -229,10 +313,27 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     float l = 0.f;
     bool ok = true;
     uint32_t sr[128];
+    // tile metadata (the listed k-blocks and their full flags), fetched one tile ahead
+    int nxt_kb0 = 0, nxt_kb1 = -1, nxt_f0 = 1, nxt_f1 = 1;
+    auto fetch_meta = [&](int j) {
+      const int e0 = rp0 + 2 * j;
+      nxt_kb0 = a.col[e0];
+      nxt_f0 = a.full[e0];
+      if (e0 + 1 < rp1) {
+        nxt_kb1 = a.col[e0 + 1];
+        nxt_f1 = a.full[e0 + 1];
+      } else {
+        nxt_kb1 = -1;
+        nxt_f1 = 1;
+      }
+    };
+    if (nT > 0) fetch_meta(0);
+    const uint64_t sl2x2 = f32x2(sl2, sl2);
     for (int j = 0; j < nT; j++) {
       const int b = j & 1;
-      const int e0 = rp0 + 2 * j;
-      const int nb = min(2, rp1 - e0);
+      const int kbs[2] = {nxt_kb0, nxt_kb1};
+      const int fls[2] = {nxt_f0, nxt_f1};
+      if (j + 1 < nT) fetch_meta(j + 1);
       // waits are made warp-uniform so that the warp-collective tcgen05 ops stay converged
       if (!__all_sync(0xffffffffu, mbar_wait(b_s(b), (j >> 1) & 1, abort_flag))) {
         ok = false;
@@ -243,29 +344,35 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
 #pragma unroll
       for (int c = 0; c < 4; c++) tmem_ld32(tS + c * 32, sr + c * 32);
       tmem_wait_ld();
-      float mx = -INFINITY;
+      // token-level mask on partial tiles, the ragged last key block and an absent second block
 #pragma unroll
       for (int h = 0; h < 2; h++) {
-        if (h < nb) {
-          const int kb = a.col[e0 + h];
-          const int k0 = kb * 64;
-          const bool need = (a.full[e0 + h] == 0) || (k0 + 64 > g.L);
-          if (need) {
+        if (kbs[h] < 0) {
+#pragma unroll
+          for (int c = 0; c < 64; c++) sr[h * 64 + c] = __float_as_uint(-INFINITY);
+        } else {
+          const int k0 = kbs[h] * 64;
+          if (fls[h] == 0 || k0 + 64 > g.L) {
 #pragma unroll
             for (int c = 0; c < 64; c++) {
               const int kk = k0 + c;
               const bool keep = (static_cast<unsigned>(kk - lo) < static_cast<unsigned>(hi - lo)) ||
-                                (kk >= g.Lv && kk < g.L);
+                                (static_cast<unsigned>(kk - g.Lv) < static_cast<unsigned>(g.T));
               if (!keep) sr[h * 64 + c] = __float_as_uint(-INFINITY);
             }
           }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 64; c++) sr[h * 64 + c] = __float_as_uint(-INFINITY);
         }
       }
+      // row maximum: 8 independent chains of 3-input max, then a small tree
+      float m8[8];
 #pragma unroll
-      for (int c = 0; c < 128; c++) mx = fmaxf(mx, __uint_as_float(sr[c]));
+      for (int i = 0; i < 8; i++) m8[i] = __uint_as_float(sr[i]);
+#pragma unroll
+      for (int c = 8; c < 128; c += 16) {
+#pragma unroll
+        for (int i = 0; i < 8; i++) m8[i] = fmax3(m8[i], __uint_as_float(sr[c + i]), __uint_as_float(sr[c + 8 + i]));
+      }
+      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
       const float mxs = mx * sl2;
       const bool need_rescale = mxs > m_use + 8.0f;
       if (__any_sync(0xffffffffu, need_rescale)) {
@@ -293,16 +400,34 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         m_use = m_new;
       }
       const float msub = (m_use == -INFINITY) ? 0.f : m_use;
-      float rs = 0.f;
+      const uint64_t nmsub2 = f32x2(-msub, -msub);
+      // P = 2^(S*scale*log2e - m): the argument as packed fp32 pairs, 2^x on the
+      // MUFU unit except for every kPolyEvery-th pair (FMA-pipe polynomial);
+      // row sum over 8 independent packed chains
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < 64; c++) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * c]), sl2, -msub));
-        const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -msub));
-        const uint32_t pk = pack_bf16x2(p0, p1);
-        rs += bf16_lo(pk) + bf16_hi(pk);
-        sr[c] = pk;
+        const uint64_t xa = ffma2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2x2, nmsub2);
+        float x0, x1;
+        unpack2(xa, x0, x1);
+        float p0, p1;
+        bool use_poly = false;
+        if constexpr (kPolyEvery > 0) use_poly = (c % kPolyStride) == kPolyStride - 1;
+        if (use_poly) {
+          poly_exp2x2(x0, x1, p0, p1);
+        } else {
+          p0 = fast_exp2(x0);
+          p1 = fast_exp2(x1);
+        }
+        acc[c & 3] = fadd2(acc[c & 3], f32x2(p0, p1));
+        sr[c] = pack_bf16x2(p0, p1);
       }
-      l += rs;
+      float s0, s1, s2, s3, s4, s5, s6, s7;
+      unpack2(acc[0], s0, s1);
+      unpack2(acc[1], s2, s3);
+      unpack2(acc[2], s4, s5);
+      unpack2(acc[3], s6, s7);
+      l += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
       tmem_st32(tS, sr);
       tmem_st32(tS + 32, sr + 32);
       tmem_wait_st();
