@@ -431,6 +431,16 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       tmem_st32(tS, sr);
       tmem_st32(tS + 32, sr + 32);
       tmem_wait_st();
+      // A parity wait on the O barrier tells "phase k done" from "not done"
+      // only when phase k-1 is known done.  The commit behind S_j covers every
+      // earlier MMA, so once S_j is ready P.V of tiles <= j-2 are done and the
+      // rescale wait above (phase j-1) is unambiguous.  The epilogue waits for
+      // phase nT-1, so phase nT-2 is confirmed here, on the last tile, before
+      // P_{nT-1} lets P.V_{nT-1} start.
+      if (j >= 1 && j == nT - 1 && !__all_sync(0xffffffffu, mbar_wait(b_o, (j - 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
       tc_fence_before();
       mbar_arrive(b_p(b));
     }

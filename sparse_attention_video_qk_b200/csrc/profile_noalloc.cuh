@@ -6,7 +6,7 @@
 
 #include <mutex>
 
-#include "profile.cuh"
+#include "profile_tc.cuh"
 #include "svg_common.cuh"
 
 namespace svg {
@@ -52,41 +52,14 @@ extern "C" svg_status svg_profile_heads_noalloc(const svg_shape* s, const svg_pa
   for (const void* ptr : ptrs)
     if (ptr && !aligned16(ptr)) return SVG_ERR_ALIGNMENT;
   const int BH = s->B * s->H;
-  // bytes of one key chunk of partial records for every head
-  const size_t per_chunk = static_cast<size_t>(BH) * kProfRows * prof_rec_floats(s->d) * sizeof(float);
-  const size_t fit = kNoAllocScratchBytes / per_chunk;
-  if (fit < 1) return SVG_ERR_CAPACITY;   // B*H*64*(4+3d)*4 bytes exceed the fixed scratch
+  // bytes of one key chunk of partial records for every head, plus the per-row error sums
+  const size_t per_chunk = static_cast<size_t>(BH) * 128 * prof_rec_floats(s->d) * sizeof(float);
+  const size_t fixed = static_cast<size_t>(BH) * kProfRows * 2 * sizeof(double);
+  if (fixed + per_chunk > kNoAllocScratchBytes) return SVG_ERR_CAPACITY;   // launches nothing
+  const size_t fit = (kNoAllocScratchBytes - fixed) / per_chunk;
   float* scratch = nullptr;
   if ((st = noalloc_scratch(&scratch)) != SVG_OK) return st;
-
-  ProfArgs a{};
-  a.g = make_geometry(s, p);
-  a.scale_log2 = scale_of(s, p) * 1.4426950408889634f;
-  a.q = qn;
-  a.k = kn;
-  a.v = v;
-  a.sample = sample_idx;
-  a.n = n;
-  const int ntiles = (a.g.L + kProfKeys - 1) / kProfKeys;
-  int nchunk = prof_chunks(BH, a.g.L);
-  if (static_cast<size_t>(nchunk) > fit) nchunk = static_cast<int>(fit);
-  a.tiles_per_chunk = (ntiles + nchunk - 1) / nchunk;
-  a.nchunk = (ntiles + a.tiles_per_chunk - 1) / a.tiles_per_chunk;   // every chunk non-empty
-  a.ws = scratch;
-  a.mse_out = mse_out;
-  a.kind_out = head_kind_out;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  dim3 grid(a.nchunk, BH);
-  if (s->d == 128) {
-    if (!set_smem(profile_partial_kernel<128>, ProfSmem<128>::BYTES)) return SVG_ERR_CUDA;
-    profile_partial_kernel<128><<<grid, kProfThreads, ProfSmem<128>::BYTES, cs>>>(a);
-    if ((st = launch_status()) != SVG_OK) return st;
-    profile_combine_kernel<128><<<BH, 256, 0, cs>>>(a);
-  } else {
-    if (!set_smem(profile_partial_kernel<64>, ProfSmem<64>::BYTES)) return SVG_ERR_CUDA;
-    profile_partial_kernel<64><<<grid, kProfThreads, ProfSmem<64>::BYTES, cs>>>(a);
-    if ((st = launch_status()) != SVG_OK) return st;
-    profile_combine_kernel<64><<<BH, 256, 0, cs>>>(a);
-  }
-  return launch_status();
+  const int nchunk = static_cast<int>(fit < static_cast<size_t>(prof_chunks(BH, s->L)) ? fit : prof_chunks(BH, s->L));
+  return launch_profile(s, p, qn, kn, v, sample_idx, n, scratch, nchunk, mse_out, head_kind_out,
+                        static_cast<cudaStream_t>(stream));
 }

@@ -10,7 +10,7 @@
 
 #include "attention.cuh"
 #include "block_index.cuh"
-#include "profile.cuh"
+#include "profile_tc.cuh"
 #include "rowmap.cuh"
 #include "svg_common.cuh"
 
@@ -139,6 +139,46 @@ svg_status launch_rowmap(const RowmapArgs& a, int D, cudaStream_t st) {
   return launch_status();
 }
 
+// Profiling: the tensor-core partial kernel over key chunks, the per-row
+// merge and the per-head choice.  `workspace` holds
+// prof_workspace_bytes(BH, L, d, max_chunks) bytes.
+svg_status launch_profile(const svg_shape* s, const svg_params* p, const uint16_t* qn, const uint16_t* kn,
+                          const uint16_t* v, const int32_t* sample_idx, int n, void* workspace, int max_chunks,
+                          float* mse_out, uint8_t* head_kind_out, cudaStream_t cs) {
+  ProfArgs a{};
+  a.g = make_geometry(s, p);
+  a.scale_log2 = scale_of(s, p) * 1.4426950408889634f;
+  a.q = qn;
+  a.sample = sample_idx;
+  a.n = n;
+  const int ntiles = (a.g.L + kProfKeys - 1) / kProfKeys;
+  const int nchunk = max(1, min(max_chunks, ntiles));
+  a.tiles_per_chunk = (ntiles + nchunk - 1) / nchunk;
+  a.nchunk = (ntiles + a.tiles_per_chunk - 1) / a.tiles_per_chunk;   // every chunk non-empty
+  a.ws = static_cast<float*>(workspace);
+  a.err = reinterpret_cast<double*>(static_cast<char*>(workspace) +
+                                    static_cast<size_t>(a.g.BH) * a.nchunk * 128 * prof_rec_floats(s->d) * sizeof(float));
+  a.mse_out = mse_out;
+  a.kind_out = head_kind_out;
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, kn, s->d, s->L, a.g.BH, 64) || !make_map(&mv, v, s->d, s->L, a.g.BH, 64)) return SVG_ERR_CUDA;
+  const dim3 grid(a.nchunk, a.g.BH), mgrid(n, a.g.BH);
+  if (s->d == 128) {
+    if (!set_smem(profile_tc_kernel<128>, ProfCfg<128>::SMEM_BYTES)) return SVG_ERR_CUDA;
+    profile_tc_kernel<128><<<grid, ProfCfg<128>::THREADS, ProfCfg<128>::SMEM_BYTES, cs>>>(mk, mv, a);
+    if (launch_status() != SVG_OK) return SVG_ERR_CUDA;
+    profile_merge_kernel<128><<<mgrid, 128, 0, cs>>>(a);
+  } else {
+    if (!set_smem(profile_tc_kernel<64>, ProfCfg<64>::SMEM_BYTES)) return SVG_ERR_CUDA;
+    profile_tc_kernel<64><<<grid, ProfCfg<64>::THREADS, ProfCfg<64>::SMEM_BYTES, cs>>>(mk, mv, a);
+    if (launch_status() != SVG_OK) return SVG_ERR_CUDA;
+    profile_merge_kernel<64><<<mgrid, 64, 0, cs>>>(a);
+  }
+  if (launch_status() != SVG_OK) return SVG_ERR_CUDA;
+  profile_choose_kernel<<<(a.g.BH + 127) / 128, 128, 0, cs>>>(a, s->d);
+  return launch_status();
+}
+
 }  // namespace
 
 // ===================================================================== ABI
@@ -235,8 +275,7 @@ int64_t svg_block_index_capacity(const svg_shape* s, const svg_params* p) {
 size_t svg_profile_workspace_size(const svg_shape* s, int n) {
   if (check_shape(s) != SVG_OK || n <= 0) return 0;
   const int BH = s->B * s->H;
-  const int nchunk = prof_chunks(BH, s->L);
-  return static_cast<size_t>(BH) * nchunk * kProfRows * prof_rec_floats(s->d) * sizeof(float);
+  return prof_workspace_bytes(BH, s->L, s->d, prof_chunks(BH, s->L));
 }
 
 svg_status svg_sync_status(void* stream) {
@@ -324,34 +363,8 @@ svg_status svg_profile_heads(const svg_shape* s, const svg_params* p, const uint
   for (const void* ptr : ptrs)
     if (ptr && !aligned16(ptr)) return SVG_ERR_ALIGNMENT;
   if (workspace_bytes < svg_profile_workspace_size(s, n)) return SVG_ERR_CAPACITY;
-  ProfArgs a{};
-  a.g = make_geometry(s, p);
-  a.scale_log2 = scale_of(s, p) * 1.4426950408889634f;
-  a.q = qn;
-  a.k = kn;
-  a.v = v;
-  a.sample = sample_idx;
-  a.n = n;
-  a.nchunk = prof_chunks(a.g.BH, a.g.L);
-  const int ntiles = (a.g.L + kProfKeys - 1) / kProfKeys;
-  a.tiles_per_chunk = (ntiles + a.nchunk - 1) / a.nchunk;
-  a.ws = static_cast<float*>(workspace);
-  a.mse_out = mse_out;
-  a.kind_out = head_kind_out;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  dim3 grid(a.nchunk, a.g.BH);
-  if (s->d == 128) {
-    if (!set_smem(profile_partial_kernel<128>, ProfSmem<128>::BYTES)) return SVG_ERR_CUDA;
-    profile_partial_kernel<128><<<grid, kProfThreads, ProfSmem<128>::BYTES, cs>>>(a);
-    if ((st = launch_status()) != SVG_OK) return st;
-    profile_combine_kernel<128><<<a.g.BH, 256, 0, cs>>>(a);
-  } else {
-    if (!set_smem(profile_partial_kernel<64>, ProfSmem<64>::BYTES)) return SVG_ERR_CUDA;
-    profile_partial_kernel<64><<<grid, kProfThreads, ProfSmem<64>::BYTES, cs>>>(a);
-    if ((st = launch_status()) != SVG_OK) return st;
-    profile_combine_kernel<64><<<a.g.BH, 256, 0, cs>>>(a);
-  }
-  return launch_status();
+  return launch_profile(s, p, qn, kn, v, sample_idx, n, workspace, prof_chunks(s->B * s->H, s->L), mse_out,
+                        head_kind_out, static_cast<cudaStream_t>(stream));
 }
 
 svg_status svg_build_block_index(const svg_shape* s, const svg_params* p, const uint8_t* head_kind,

@@ -46,12 +46,15 @@ CASES = {
     "tiny64": W.small_workload(d=64, H=2, F=1, Hs=2, Ws=3, T=5, w=0, r=1, n_samples=4, bq=64),
     # several frames per key tile (S = 20), bq = 64
     "smallS": W.small_workload(d=64, H=4, F=9, Hs=4, Ws=5, T=3, w=2, r=4, n_samples=16, bq=64),
+    # the same grid with d = 128, and without text (the last key tile's second half is past L)
+    "smallS128": W.small_workload(d=128, H=4, F=9, Hs=4, Ws=5, T=3, w=2, r=4, n_samples=16, bq=128),
+    "smallS_T0": W.small_workload(d=64, H=4, F=9, Hs=4, Ws=5, T=0, w=2, r=4, n_samples=16, bq=64),
     # one frame: the temporal layout is the identity
     "oneframe": W.small_workload(d=128, H=2, F=1, Hs=12, Ws=20, T=7, w=0, r=30, n_samples=8),
     # wide windows that reduce to dense
     "wide": W.small_workload(d=64, H=2, F=5, Hs=6, Ws=7, T=9, w=4, r=41, n_samples=8),
 }
-FULL_ROW_CASES = ("cfg0", "ragged128", "tiny64", "smallS", "oneframe", "wide")
+FULL_ROW_CASES = ("cfg0", "ragged128", "tiny64", "smallS", "smallS128", "smallS_T0", "oneframe", "wide")
 
 
 def pb_of(wl):
@@ -177,7 +180,7 @@ def test_block_index_capacity_overflow_is_reported():
 
 # --------------------------------------------------------------- profiling
 
-@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "smallS", "ragged128", "cfg3"])
+@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "smallS", "smallS128", "smallS_T0", "ragged128", "cfg3"])
 def test_profile_choices_bit_exact(key):
     wl, inp, qn, kn = case(key)
     pb = pb_of(wl)
@@ -224,7 +227,8 @@ def run_sparse(wl, qn, kn, v, kinds, want_lse=False):
     return out, lse
 
 
-@pytest.mark.parametrize("key", ["cfg0", "ragged128", "tiny64", "smallS", "oneframe", "wide", "cfg1", "cfg2"])
+@pytest.mark.parametrize("key", ["cfg0", "ragged128", "tiny64", "smallS", "smallS128", "smallS_T0", "oneframe", "wide",
+                                 "cfg1", "cfg2"])
 @pytest.mark.parametrize("kinds_mode", ["mixed", "spatial", "temporal"])
 def test_attention_parity(key, kinds_mode):
     wl, inp, qn, kn = case(key)
