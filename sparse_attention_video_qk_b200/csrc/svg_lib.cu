@@ -126,16 +126,33 @@ bool set_smem(K kernel, int bytes) {
 
 // ------------------------------------------------------------- rowmap ----
 
-svg_status launch_rowmap(const RowmapArgs& a, int D, cudaStream_t st) {
-  const int64_t rows = static_cast<int64_t>(a.g.BH) * a.g.L * a.ntensor;
-  const int rows_per_block = 8 * (32 / (D / 8)) * 4;   // warps * rows per step * steps
-  int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
-  if (blocks > kNumSMs * 8) blocks = kNumSMs * 8;
-  if (blocks < 1) blocks = 1;
-  if (D == 128)
-    rowmap_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
-  else
-    rowmap_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
+svg_status launch_rowmap(RowmapArgs a, int D, cudaStream_t st) {
+  a.divF = make_fastdiv(a.g.F);
+  a.divS = make_fastdiv(a.g.S);
+  a.divWs = make_fastdiv(a.g.Ws);
+  const int unit_rows = 8 * (32 / (D / 8)) * kRowmapSteps * kRowmapUnitSteps;
+  const int64_t nunits = static_cast<int64_t>(a.ntensor) * a.g.BH * ((a.g.L + unit_rows - 1) / unit_rows);
+  if (nunits > INT32_MAX) return SVG_ERR_UNSUPPORTED;
+  int64_t blocks = static_cast<int64_t>(kNumSMs) * 4;      // resident capacity at 4 blocks per SM
+  if (blocks > nunits) blocks = nunits;
+  const dim3 grid(static_cast<unsigned>(blocks));
+  const bool staged = a.norm_tensors > 0 && a.rope_floats <= kRopeSmemFloats;
+  const int smem = staged ? a.rope_floats * 4 : 0;
+  if (D == 128) {
+    if (staged) {
+      if (!set_smem(rowmap_kernel<128, true>, smem)) return SVG_ERR_CUDA;
+      rowmap_kernel<128, true><<<grid, 256, smem, st>>>(a);
+    } else {
+      rowmap_kernel<128, false><<<grid, 256, 0, st>>>(a);
+    }
+  } else {
+    if (staged) {
+      if (!set_smem(rowmap_kernel<64, true>, smem)) return SVG_ERR_CUDA;
+      rowmap_kernel<64, true><<<grid, 256, smem, st>>>(a);
+    } else {
+      rowmap_kernel<64, false><<<grid, 256, 0, st>>>(a);
+    }
+  }
   return launch_status();
 }
 
@@ -325,6 +342,7 @@ svg_status svg_qknorm_rope_layout(const svg_shape* s, const svg_params* p, int f
   a.gamma[0] = gamma_q;
   a.gamma[1] = gamma_k;
   a.rope = reinterpret_cast<const float2*>(rope_table);
+  a.rope_floats = (flags & SVG_NORM_ROPE) ? static_cast<int>(svg_rope_table_size(s, p)) : 0;
   a.kind = head_kind;
   a.eps = p->eps;
   a.split0 = p->rope_split[0];
