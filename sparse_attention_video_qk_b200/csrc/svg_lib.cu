@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "attention.cuh"
+#include "attention2.cuh"
 #include "block_index.cuh"
 #include "profile_tc.cuh"
 #include "rowmap.cuh"
@@ -428,8 +429,20 @@ svg_status svg_block_sparse_attn(const svg_shape* s, const svg_params* p, const 
   if (!make_map(&mq, q, s->d, s->L, a.g.BH, 128) || !make_map(&mk, k, s->d, s->L, a.g.BH, 64) ||
       !make_map(&mv, v, s->d, s->L, a.g.BH, 64))
     return SVG_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(a.g.BH) * static_cast<unsigned>(a.g.nqb);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (a.g.bq == 128) {
+    // two 128-row query tiles per CTA share every K/V tile
+    const unsigned grid = static_cast<unsigned>(a.g.BH) * static_cast<unsigned>((a.g.nqb + 1) / 2);
+    if (s->d == 128) {
+      if (!set_smem(attn2_kernel<128>, Attn2Cfg<128>::SMEM_BYTES)) return SVG_ERR_CUDA;
+      attn2_kernel<128><<<grid, Attn2Cfg<128>::THREADS, Attn2Cfg<128>::SMEM_BYTES, cs>>>(mq, mk, mv, a);
+    } else {
+      if (!set_smem(attn2_kernel<64>, Attn2Cfg<64>::SMEM_BYTES)) return SVG_ERR_CUDA;
+      attn2_kernel<64><<<grid, Attn2Cfg<64>::THREADS, Attn2Cfg<64>::SMEM_BYTES, cs>>>(mq, mk, mv, a);
+    }
+    return launch_status();
+  }
+  const unsigned grid = static_cast<unsigned>(a.g.BH) * static_cast<unsigned>(a.g.nqb);
   if (s->d == 128) {
     if (!set_smem(attn_kernel<128>, AttnCfg<128>::SMEM_BYTES)) return SVG_ERR_CUDA;
     attn_kernel<128><<<grid, AttnCfg<128>::THREADS, AttnCfg<128>::SMEM_BYTES, cs>>>(mq, mk, mv, a);
