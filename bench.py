@@ -281,7 +281,10 @@ def run_gpu(args, rank, world, local_rank):
 
     pk, pk_src = peaks()
     attn_tflops = flops / (stage_ms["attention"] * 1e-3) / 1e12
-    traffic = traffic_from_profile("attention.cuh", "attention_hunyuan_cfg3.md")
+    # svg_block_sparse_attn runs the two-query-tile kernel for 128-row tiles
+    attn_src, attn_name = (("attention2.cuh", f"attn2_kernel<{wl.d}>") if wl.bq == 128
+                           else ("attention.cuh", f"attn_kernel<{wl.d}>"))
+    traffic = traffic_from_profile(attn_src, "attention_hunyuan_cfg3.md") if args.config == 3 else None
     d, L, BH = wl.d, wl.L, wl.B * wl.H
     stage_bytes = {"qknorm_rope": 8.0 * BH * L * d, "layout": 12.0 * BH * L * d, "inverse_layout": 4.0 * BH * L * d,
                    "profile": 4.0 * BH * L * d}
@@ -315,7 +318,7 @@ def run_gpu(args, rank, world, local_rank):
         "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "stage_gbs": {k: round(stage_bytes[k] / (stage_ms[k] * 1e-3) / 1e9, 1) for k in stage_bytes},
         "roofline": {
-            "kernel": "attn_kernel<128> (svg_block_sparse_attn)",
+            "kernel": f"{attn_name} (svg_block_sparse_attn)",
             "bound": "tensor",
             "achieved": round(attn_tflops, 2),
             "peak": pk["bf16_tflops_sustained"],
@@ -440,7 +443,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--config", type=int, default=3)
-    ap.add_argument("--cpu-rows", type=int, default=1920)
+    ap.add_argument("--cpu-rows", type=int, default=9600)
     ap.add_argument("--ref-rows", type=int, default=960)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -105,8 +105,9 @@ svg_status svg_qknorm_rope_layout(const svg_shape* shape, const svg_params* para
 /* Stage 2: online profiling.
  * For every (b, h) and each of the n sampled video tokens sample_idx[0..n) (device
  * int32, the same rows for every head, 1 <= n <= 64): the dense, the spatial-masked and
- * the temporal-masked attention outputs of that query row (fp32 softmax, P split into
- * two bf16 terms for the tensor-core products).  Per head
+ * the temporal-masked attention outputs of that query row (fp32 softmax; P rounded to
+ * bf16 for the tensor-core P.V, and the row sums taken from the same rounded values,
+ * so each output stays a weighted average).  Per head
  *   MSE_m = mean over the n rows and d columns of (O_m - O_dense)^2,  m in {spatial, temporal}
  * and head_kind_out[b*H+h] = SPATIAL if MSE_spatial <= MSE_temporal else TEMPORAL.
  * qn, kn: device bf16 [B,H,L,d] after stage 1, frame-major order; v: device bf16.
@@ -128,9 +129,10 @@ svg_status svg_profile_heads(const svg_shape* shape, const svg_params* params,
  * the workspace) and allocates nothing: its scratch is a fixed 16 MiB device
  * array inside the library, which every GPU that loads the library holds until
  * the process exits.
- *   - Size limit: one key chunk of partial results takes B*H*64*(4+3d)*4 bytes;
- *     if that exceeds 16 MiB (B*H > 168 at d=128, > 334 at d=64) the call
- *     returns SVG_ERR_CAPACITY and launches nothing.  Otherwise it splits the
+ *   - Size limit: one key chunk of partial results takes B*H*128*(3+2d)*4 bytes
+ *     and the per-row error sums B*H*64*2*8 bytes; if together they exceed
+ *     16 MiB (B*H > 125 at d=128, > 246 at d=64) the call returns
+ *     SVG_ERR_CAPACITY and launches nothing.  Otherwise it splits the
  *     keys into as many chunks as fit (at most as many as svg_profile_heads).
  *   - Set-up: the first call on each device looks up the scratch's device
  *     address (cudaGetSymbolAddress, with that device current) and caches it;

@@ -67,12 +67,9 @@ __device__ __forceinline__ uint64_t fma_f2(uint64_t a, uint64_t b, uint64_t c) {
 #ifndef SVG_ROWMAP_STEPS
 #define SVG_ROWMAP_STEPS 4
 #endif
-#ifndef SVG_ROWMAP_BLOCKS_PER_SM
-#define SVG_ROWMAP_BLOCKS_PER_SM 8
-#endif
 constexpr int kRowmapSteps = SVG_ROWMAP_STEPS;            // row steps each warp keeps in flight
 constexpr int kRowmapUnitSteps = 4;                       // block iterations per work unit
-constexpr int kRowmapBlocksPerSM = SVG_ROWMAP_BLOCKS_PER_SM;
+constexpr int kRowmapBlocksPerSM = 4;                     // resident blocks of 256 threads per SM
 
 constexpr int kRopeSmemFloats = 24576;  // 96 KB: tables up to this size are staged in shared memory
 
@@ -96,7 +93,7 @@ struct RowmapArgs {
 // STAGED: the RoPE table is copied into shared memory (dynamic, rope_floats * 4
 // bytes); otherwise it is read through the read-only data cache.
 template <int D, bool STAGED>
-__global__ void __launch_bounds__(256, 4) rowmap_kernel(const RowmapArgs a) {
+__global__ void __launch_bounds__(256, kRowmapBlocksPerSM) rowmap_kernel(const RowmapArgs a) {
   constexpr int LPR = D / 8;       // lanes per row
   constexpr int RPW = 32 / LPR;    // rows per warp step
   constexpr int U = kRowmapSteps;  // warp steps in flight

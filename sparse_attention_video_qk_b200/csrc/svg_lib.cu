@@ -134,7 +134,7 @@ svg_status launch_rowmap(RowmapArgs a, int D, cudaStream_t st) {
   const int unit_rows = 8 * (32 / (D / 8)) * kRowmapSteps * kRowmapUnitSteps;
   const int64_t nunits = static_cast<int64_t>(a.ntensor) * a.g.BH * ((a.g.L + unit_rows - 1) / unit_rows);
   if (nunits > INT32_MAX) return SVG_ERR_UNSUPPORTED;
-  int64_t blocks = static_cast<int64_t>(kNumSMs) * 4;      // resident capacity at 4 blocks per SM
+  int64_t blocks = static_cast<int64_t>(kNumSMs) * kRowmapBlocksPerSM;   // the resident capacity
   if (blocks > nunits) blocks = nunits;
   const dim3 grid(static_cast<unsigned>(blocks));
   const bool staged = a.norm_tensors > 0 && a.rope_floats <= kRopeSmemFloats;

@@ -110,3 +110,20 @@ def test_host_side_argument_errors(L):
                                None) == C.SVG_ERR_INVALID_ARG
     assert L.svg_profile_heads(ctypes.byref(sh), ctypes.byref(pr), p, p, p, p, 16, p, 16, None, p,
                                None) == C.SVG_ERR_CAPACITY
+
+
+def test_noalloc_capacity_limit(L):
+    """The no-alloc profiling entry rejects shapes whose one key chunk of
+    partials does not fit its 16 MiB scratch, before any CUDA call."""
+    p = ctypes.c_void_p(16)
+    for wl_idx, heads in ((2, 126), (1, 247)):          # d = 128: B*H > 125; d = 64: B*H > 246
+        pb = api.Problem.from_workload(W.CONFIGS[wl_idx])
+        sh, pr = pb.c_shape(), pb.c_params()
+        big = C.SvgShape(1, heads, sh.L, sh.d, sh.F, sh.Hs, sh.Ws, sh.text_len)
+        per_chunk = heads * 128 * (3 + 2 * sh.d) * 4 + heads * 64 * 2 * 8
+        assert per_chunk > 16 << 20
+        assert (heads - 1) * 128 * (3 + 2 * sh.d) * 4 + (heads - 1) * 64 * 2 * 8 <= 16 << 20
+        assert L.svg_profile_heads_noalloc(ctypes.byref(big), ctypes.byref(pr), p, p, p, p, 64, None, p,
+                                           None) == C.SVG_ERR_CAPACITY
+        assert L.svg_profile_heads_noalloc(ctypes.byref(sh), ctypes.byref(pr), p, p, p, p, 65, None, p,
+                                           None) == C.SVG_ERR_INVALID_ARG

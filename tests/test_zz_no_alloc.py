@@ -47,7 +47,7 @@ def test_noalloc_matches_workspace_entry_point_twice(cfg):
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
-    # one key chunk of partials for 200 heads at d = 128 needs 200*64*388*4 B > 16 MiB
+    # one key chunk of partials for 200 heads at d = 128 needs 200*128*259*4 B > 16 MiB
     wl = W.small_workload(d=128, H=200, F=2, Hs=2, Ws=4, T=0, n_samples=4)
     pb = svg.Problem.from_workload(wl)
     x = torch.zeros(1, 200, wl.L, 128, dtype=torch.bfloat16, device="cuda")
