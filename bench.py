@@ -3,7 +3,7 @@
 Default workload: HunyuanVideo 720p 5 s shape (B=1, H=24, d=128, 33 latent
 frames of 45x80 = 118,800 video tokens + 256 text tokens), one full step per
 iteration: QK-Norm + 3D RoPE -> online profiling -> block index -> layout
-transform -> block-sparse attention -> inverse layout.
+transform -> block-sparse attention with the inverse layout in its epilogue.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--sweep]
 
@@ -172,7 +172,7 @@ def run_gpu(args, rank, world, local_rank):
     P = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
     def stage_calls():
-        """The step as its six C-ABI calls (same as svg_attention_step)."""
+        """The step as its five C-ABI calls (the same calls svg_attention_step makes)."""
         b = buf
         return [
             ("qknorm_rope", lambda: lib.svg_qknorm_rope_layout(ctypes.byref(sh), ctypes.byref(pr), 1, P(q), P(k), None,
@@ -186,14 +186,15 @@ def run_gpu(args, rank, world, local_rank):
             ("layout", lambda: lib.svg_qknorm_rope_layout(ctypes.byref(sh), ctypes.byref(pr), 2, P(b.qn), P(b.kn),
                                                           P(v), None, None, None, P(b.kinds), P(b.qp), P(b.kp),
                                                           P(b.vp), cs)),
-            ("attention", lambda: lib.svg_block_sparse_attn(ctypes.byref(sh), ctypes.byref(pr), P(b.qp), P(b.kp),
-                                                            P(b.vp), P(b.kinds), P(b.row_ptr), P(b.col), P(b.full),
-                                                            P(b.op), None, cs)),
-            ("inverse_layout", lambda: lib.svg_inverse_layout(ctypes.byref(sh), P(b.kinds), P(b.op), P(b.out), cs)),
+            # attention with the inverse layout in its epilogue: writes `out` in model order
+            ("attention", lambda: lib.svg_block_sparse_attn_model_order(
+                ctypes.byref(sh), ctypes.byref(pr), P(b.qp), P(b.kp), P(b.vp), P(b.kinds), P(b.row_ptr),
+                P(b.col), P(b.full), P(b.out), None, cs)),
         ]
 
     calls = stage_calls()
-    launches_per_step = 1 + 2 + 3 + 1 + 1 + 1
+    # kernels per stage: rowmap; profile_tc + merge + choose; count + scan + fill; rowmap; attention
+    launches_per_step = 1 + 3 + 3 + 1 + 1
 
     def one_step(events=None):
         for i, (name, fn) in enumerate(calls):
@@ -286,7 +287,7 @@ def run_gpu(args, rank, world, local_rank):
                            else ("attention.cuh", f"attn_kernel<{wl.d}>"))
     traffic = traffic_from_profile(attn_src, "attention_hunyuan_cfg3.md") if args.config == 3 else None
     d, L, BH = wl.d, wl.L, wl.B * wl.H
-    stage_bytes = {"qknorm_rope": 8.0 * BH * L * d, "layout": 12.0 * BH * L * d, "inverse_layout": 4.0 * BH * L * d,
+    stage_bytes = {"qknorm_rope": 8.0 * BH * L * d, "layout": 12.0 * BH * L * d,
                    "profile": 4.0 * BH * L * d}
     line = {
         "metric": METRIC,
@@ -340,6 +341,92 @@ def run_gpu(args, rank, world, local_rank):
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_rows)
     return line
+
+
+# ------------------------------------------------------ sparsity sweep --
+
+def token_density(wl, kind):
+    """Kept (query, key) pairs over video query rows against all L keys, from
+    the masks' closed forms (text keys always kept)."""
+    F, S, T, L = wl.F, wl.S, wl.T, wl.L
+    if kind == W.SPATIAL:
+        f = np.arange(F)
+        frames = np.minimum(f + wl.w, F - 1) - np.maximum(f - wl.w, 0) + 1
+        kept = float(np.sum(frames * S + T)) * S
+    else:
+        s = np.arange(S)
+        locs = np.minimum(s + wl.r, S - 1) - np.maximum(s - wl.r, 0) + 1
+        kept = float(np.sum(locs * F + T)) * F
+    return kept / (float(wl.Lv) * L)
+
+
+def run_sweep(args):
+    """Forced-kind sweep at the config-3 shape: every head spatial with
+    w in {0,1,2,4,8}, then every head temporal (layout applied) with r in
+    {32,...,1800}; attention time against dense on the same inputs."""
+    import torch
+
+    import sparse_attention_video_qk_b200 as svg
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    base = W.CONFIGS[4]
+    pb0 = svg.Problem.from_workload(base)
+    g = torch.Generator(device=device).manual_seed(base.seed)
+    shp = (base.B, base.H, base.L, base.d)
+    q, k, v = (torch.randn(shp, generator=g, device=device).to(torch.bfloat16) for _ in range(3))
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+
+    def time_attn(pb, qq, kk, vv, kinds, rp, col, full, reps):
+        for _ in range(args.warmup):
+            svg.block_sparse_attn(pb, qq, kk, vv, kinds, rp, col, full, out=out)
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            svg.block_sparse_attn(pb, qq, kk, vv, kinds, rp, col, full, out=out)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        svg.sync_status()
+        return statistics.median(ms)
+
+    dk = torch.full((base.B * base.H,), svg.DENSE, dtype=torch.uint8, device=device)
+    rp, col, full = svg.build_block_index(pb0, dk, svg.block_index_capacity(pb0))
+    dense_ms = time_attn(pb0, q, k, v, dk, rp, col, full, max(3, args.steps // 4))
+    dense_flops = kept_tile_flops(rp.cpu().numpy(), col[: int(rp[-1])].cpu().numpy(), base)
+    points = []
+    with ClockSampler(0) as clk:
+        clk.start()
+        for label, wl in W.sweep_points():
+            pb = svg.Problem.from_workload(wl)
+            kind = wl.forced_kinds[0]
+            kinds = torch.full((wl.B * wl.H,), kind, dtype=torch.uint8, device=device)
+            qq, kk, vv = svg.layout(pb, q, k, v, kinds) if kind == W.TEMPORAL else (q, k, v)
+            rp, col, full = svg.build_block_index(pb, kinds, svg.block_index_capacity(pb))
+            ms = time_attn(pb, qq, kk, vv, kinds, rp, col, full, args.steps)
+            nnz = int(rp[-1])
+            flops = kept_tile_flops(rp.cpu().numpy(), col[:nnz].cpu().numpy(), wl)
+            td = token_density(wl, kind)
+            points.append({
+                "point": label, "ms": round(ms, 3), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+                "kept_tile_tflop": round(flops / 1e12, 3), "token_density": round(td, 4),
+                "tile_density": round(flops / dense_flops, 4),
+                "speedup_vs_dense": round(dense_ms / ms, 2),
+                "theoretical_tiles": round(dense_flops / flops, 2),
+                "theoretical_tokens": round(1.0 / td, 2)})
+            del qq, kk, vv
+        clk.stop()
+    pk, pk_src = peaks()
+    return {"sweep": "forced-kind sparsity sweep at the HunyuanVideo 720p 5 s shape",
+            "steps_per_point": args.steps, "warmup": args.warmup, "statistic": "median CUDA-event ms",
+            "dense": {"ms": round(dense_ms, 3), "tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 1),
+                      "tflop": round(dense_flops / 1e12, 3)},
+            "peak_bf16_sustained": pk["bf16_tflops_sustained"], "peak_source": pk_src,
+            "points": points, "clocks": clk.summary(),
+            "data": "synthetic N(0,1) bf16 Q/K/V, head kinds forced"}
 
 
 # ---------------------------------------------------------- oracle (CPU) --
@@ -443,10 +530,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--config", type=int, default=3)
-    ap.add_argument("--cpu-rows", type=int, default=9600)
+    ap.add_argument("--cpu-rows", type=int, default=14400)
     ap.add_argument("--ref-rows", type=int, default=960)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="forced-kind sparsity sweep (one GPU); prints one JSON line with every point")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -455,6 +544,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if world != args.gpus:
         world = max(world, 1)
+    if args.sweep:
+        if rank == 0:
+            print(json.dumps(run_sweep(args)), flush=True)
+        return
     if args.impl == "reference":
         line = run_reference(args, rank)
         if line is not None:

@@ -179,6 +179,21 @@ svg_status svg_block_sparse_attn(const svg_shape* shape, const svg_params* param
                                  const int32_t* col, const uint8_t* full,
                                  uint16_t* out, float* lse_out, void* stream);
 
+/* Stage 4 with stage 5 fused into its epilogue: as svg_block_sparse_attn, but
+ * every output row (and LSE entry) is stored at its model-order position --
+ * rows of temporal heads go from s*F+f back to f*S+s, all other rows stay -- so
+ * the separate inverse-layout pass and its read and write of O disappear.
+ * The pages describe the inverse transform as a step of its own ("Sparse
+ * VideoGen" WeChat article, "硬件高效的 Layout Transformation"); fusing it is
+ * this library's choice.  out: device bf16 [B,H,L,d] in model order;
+ * lse_out: device fp32 [B,H,L] in model order, or NULL.  Other arguments and
+ * errors as for svg_block_sparse_attn. */
+svg_status svg_block_sparse_attn_model_order(const svg_shape* shape, const svg_params* params,
+                                             const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                             const uint8_t* head_kind, const int32_t* row_ptr,
+                                             const int32_t* col, const uint8_t* full,
+                                             uint16_t* out, float* lse_out, void* stream);
+
 /* Stage 5: inverse of the layout transform (temporal heads: row s*F+f -> f*S+s).
  * src, dst: device bf16 [B,H,L,d]; head_kind: device uint8 [B*H]. */
 svg_status svg_inverse_layout(const svg_shape* shape, const uint8_t* head_kind,
@@ -187,8 +202,11 @@ svg_status svg_inverse_layout(const svg_shape* shape, const uint8_t* head_kind,
 /* The five stages in order on one stream (profiling skipped when
  * head_kind_in != NULL, whose kinds are then used).  All buffers are device
  * memory owned by the caller:
- *   qn, kn, qp, kp, vp: bf16 [B,H,L,d] intermediates; op: bf16 [B,H,L,d] output
- *   in the head's layout; out: bf16 [B,H,L,d] final output in model order;
+ *   qn, kn, qp, kp, vp: bf16 [B,H,L,d] intermediates;
+ *   op: bf16 [B,H,L,d] attention output in the head's layout, or NULL -- with
+ *   NULL, the attention writes `out` in model order directly
+ *   (svg_block_sparse_attn_model_order) and no inverse pass runs;
+ *   out: bf16 [B,H,L,d] final output in model order;
  *   head_kind_out: uint8 [B*H]; mse_out: fp32 [B*H*2] or NULL;
  *   row_ptr/col/full: block index with `capacity` entries;
  *   workspace: svg_profile_workspace_size(shape, n) bytes. */

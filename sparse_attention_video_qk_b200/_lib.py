@@ -43,6 +43,7 @@ SIGNATURES = {
     "svg_profile_heads_noalloc": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp]),
     "svg_build_block_index": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _i64, _vp]),
     "svg_block_sparse_attn": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "svg_block_sparse_attn_model_order": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "svg_inverse_layout": (_i32, [_SP, _vp, _vp, _vp, _vp]),
     "svg_attention_step": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
                                   _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,

@@ -196,14 +196,18 @@ def build_block_index(pb: Problem, kinds, capacity=None, out=None, stream=None):
     return row_ptr, col, full
 
 
-def block_sparse_attn(pb: Problem, q, k, v, kinds, row_ptr, col, full, out=None, want_lse=False, stream=None):
+def block_sparse_attn(pb: Problem, q, k, v, kinds, row_ptr, col, full, out=None, want_lse=False, stream=None,
+                      model_order=False):
+    """Stage 4.  out (and lse) in the head's layout, or with model_order=True
+    in model order (stage 5 fused into the epilogue)."""
     sh, pr = pb.c_shape(), pb.c_params()
     if out is None:
         out = torch.empty_like(q)
     lse = torch.empty(pb.B, pb.H, pb.L, dtype=torch.float32, device=q.device) if want_lse else None
-    st = lib().svg_block_sparse_attn(ctypes.byref(sh), ctypes.byref(pr), _p(q), _p(k), _p(v), _p(kinds),
-                                     _p(row_ptr), _p(col), _p(full), _p(out), _p(lse), _stream(stream))
-    check(st, "svg_block_sparse_attn")
+    name = "svg_block_sparse_attn_model_order" if model_order else "svg_block_sparse_attn"
+    st = getattr(lib(), name)(ctypes.byref(sh), ctypes.byref(pr), _p(q), _p(k), _p(v), _p(kinds),
+                              _p(row_ptr), _p(col), _p(full), _p(out), _p(lse), _stream(stream))
+    check(st, name)
     return (out, lse) if want_lse else out
 
 
@@ -219,14 +223,18 @@ def inverse_layout(pb: Problem, kinds, src, out=None, stream=None):
 # --------------------------------------------------------------- full step --
 
 class StepBuffers:
-    """Device buffers of one step, allocated once for a Problem and reused."""
+    """Device buffers of one step, allocated once for a Problem and reused.
+    With head_layout_out=True the step also keeps the attention output in the
+    head's layout (`op`) and runs the inverse layout as a pass of its own;
+    otherwise (default) the attention writes `out` in model order directly."""
 
-    def __init__(self, pb: Problem, n_samples: int, device="cuda"):
+    def __init__(self, pb: Problem, n_samples: int, device="cuda", head_layout_out=False):
         shp = (pb.B, pb.H, pb.L, pb.d)
         mk = lambda: torch.empty(shp, dtype=torch.bfloat16, device=device)
         self.pb = pb
         self.n = n_samples
-        self.qn, self.kn, self.qp, self.kp, self.vp, self.op, self.out = (mk() for _ in range(7))
+        self.qn, self.kn, self.qp, self.kp, self.vp, self.out = (mk() for _ in range(6))
+        self.op = mk() if head_layout_out else None
         self.kinds = torch.empty(pb.B * pb.H, dtype=torch.uint8, device=device)
         self.mse = torch.empty(pb.B * pb.H, 2, dtype=torch.float32, device=device)
         self.capacity = block_index_capacity(pb)

@@ -64,9 +64,19 @@ struct AttnArgs {
   const int32_t* row_ptr;        // [BH*nqb + 1]
   const int32_t* col;            // [nnz]
   const uint8_t* full;           // [nnz]
-  uint16_t* out;                 // [BH, L, D] bf16, head's layout
+  uint16_t* out;                 // [BH, L, D] bf16, head's layout (or model order, see below)
   float* lse;                    // [BH, L] or null
+  int model_order;               // 1: rows of temporal heads are stored back in frame-major order
 };
+
+// Row of `out` / `lse` that receives query row `row` (given in the head's
+// layout): the row itself, or, with model_order, its frame-major position --
+// the inverse layout transform (temporal heads: s*F+f -> f*S+s; text rows stay).
+__device__ __forceinline__ int out_row(const Geometry& g, int model_order, int kind, int row) {
+  if (!model_order || kind != SVG_HEAD_TEMPORAL || row >= g.Lv) return row;
+  const int s = row / g.F, f = row - s * g.F;
+  return f * g.S + s;
+}
 
 // 2^x with the MUFU.EX2 unit (PTX ex2.approx.ftz.f32); 2^-inf = 0.
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -449,7 +459,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     if (ok && nT > 0 && __all_sync(0xffffffffu, mbar_wait(b_o, (nT - 1) & 1, abort_flag))) {
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      uint16_t* orow = a.out + (static_cast<int64_t>(bh) * g.L + row) * D;
+      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row(g, a.model_order, kind, row);
+      uint16_t* orow = a.out + orow_i * D;
 #pragma unroll
       for (int c = 0; c < D / 32; c++) {
         uint32_t o[32];
@@ -468,14 +479,12 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           }
         }
       }
-      if (row_ok && a.lse) {
-        a.lse[static_cast<int64_t>(bh) * g.L + row] =
-            (l > 0.f) ? (m_use * 0.69314718055994531f + logf(l)) : -INFINITY;
-      }
+      if (row_ok && a.lse) a.lse[orow_i] = (l > 0.f) ? (m_use * 0.69314718055994531f + logf(l)) : -INFINITY;
     } else if (ok && nT == 0 && row_ok) {
-      uint4* dst = reinterpret_cast<uint4*>(a.out + (static_cast<int64_t>(bh) * g.L + row) * D);
+      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row(g, a.model_order, kind, row);
+      uint4* dst = reinterpret_cast<uint4*>(a.out + orow_i * D);
       for (int v = 0; v < D / 8; v++) dst[v] = make_uint4(0, 0, 0, 0);
-      if (a.lse) a.lse[static_cast<int64_t>(bh) * g.L + row] = -INFINITY;
+      if (a.lse) a.lse[orow_i] = -INFINITY;
     }
   }
   tc_fence_before();

@@ -440,7 +440,8 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
     if (ok && nT > 0 && __all_sync(0xffffffffu, mbar_wait(b_o(w), (nT - 1) & 1, abort_flag))) {
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      uint16_t* orow = a.out + (static_cast<int64_t>(bh) * g.L + row) * D;
+      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row(g, a.model_order, kind, row);
+      uint16_t* orow = a.out + orow_i * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; c++) {
         uint32_t o[32];
@@ -459,14 +460,12 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
           }
         }
       }
-      if (row_ok && a.lse) {
-        a.lse[static_cast<int64_t>(bh) * g.L + row] =
-            (l > 0.f) ? (m_use * 0.69314718055994531f + logf(l)) : -INFINITY;
-      }
+      if (row_ok && a.lse) a.lse[orow_i] = (l > 0.f) ? (m_use * 0.69314718055994531f + logf(l)) : -INFINITY;
     } else if (ok && nT == 0 && row_ok) {
-      uint4* dst = reinterpret_cast<uint4*>(a.out + (static_cast<int64_t>(bh) * g.L + row) * D);
+      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row(g, a.model_order, kind, row);
+      uint4* dst = reinterpret_cast<uint4*>(a.out + orow_i * D);
       for (int v = 0; v < D / 8; v++) dst[v] = make_uint4(0, 0, 0, 0);
-      if (a.lse) a.lse[static_cast<int64_t>(bh) * g.L + row] = -INFINITY;
+      if (a.lse) a.lse[orow_i] = -INFINITY;
     }
   }
   tc_fence_before();

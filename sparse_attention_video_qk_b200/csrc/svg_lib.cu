@@ -404,10 +404,12 @@ svg_status svg_build_block_index(const svg_shape* s, const svg_params* p, const 
   return launch_status();
 }
 
-svg_status svg_block_sparse_attn(const svg_shape* s, const svg_params* p, const uint16_t* q, const uint16_t* k,
-                                 const uint16_t* v, const uint8_t* head_kind, const int32_t* row_ptr,
-                                 const int32_t* col, const uint8_t* full, uint16_t* out, float* lse_out,
-                                 void* stream) {
+// Block-sparse attention; model_order = 1 also applies the inverse layout
+// (temporal heads' rows are stored back in frame-major order).
+static svg_status attention_launch(const svg_shape* s, const svg_params* p, const uint16_t* q, const uint16_t* k,
+                                   const uint16_t* v, const uint8_t* head_kind, const int32_t* row_ptr,
+                                   const int32_t* col, const uint8_t* full, uint16_t* out, float* lse_out,
+                                   int model_order, void* stream) {
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if ((st = check_params(s, p, true)) != SVG_OK) return st;
@@ -425,6 +427,7 @@ svg_status svg_block_sparse_attn(const svg_shape* s, const svg_params* p, const 
   a.full = full;
   a.out = out;
   a.lse = lse_out;
+  a.model_order = model_order;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, s->d, s->L, a.g.BH, 128) || !make_map(&mk, k, s->d, s->L, a.g.BH, 64) ||
       !make_map(&mv, v, s->d, s->L, a.g.BH, 64))
@@ -453,6 +456,20 @@ svg_status svg_block_sparse_attn(const svg_shape* s, const svg_params* p, const 
   return launch_status();
 }
 
+svg_status svg_block_sparse_attn(const svg_shape* s, const svg_params* p, const uint16_t* q, const uint16_t* k,
+                                 const uint16_t* v, const uint8_t* head_kind, const int32_t* row_ptr,
+                                 const int32_t* col, const uint8_t* full, uint16_t* out, float* lse_out,
+                                 void* stream) {
+  return attention_launch(s, p, q, k, v, head_kind, row_ptr, col, full, out, lse_out, 0, stream);
+}
+
+svg_status svg_block_sparse_attn_model_order(const svg_shape* s, const svg_params* p, const uint16_t* q,
+                                             const uint16_t* k, const uint16_t* v, const uint8_t* head_kind,
+                                             const int32_t* row_ptr, const int32_t* col, const uint8_t* full,
+                                             uint16_t* out, float* lse_out, void* stream) {
+  return attention_launch(s, p, q, k, v, head_kind, row_ptr, col, full, out, lse_out, 1, stream);
+}
+
 svg_status svg_attention_step(const svg_shape* s, const svg_params* p, const uint16_t* q, const uint16_t* k,
                               const uint16_t* v, const float* gamma_q, const float* gamma_k, const float* rope_table,
                               const int32_t* sample_idx, int n, const uint8_t* head_kind_in, uint16_t* qn,
@@ -475,6 +492,8 @@ svg_status svg_attention_step(const svg_shape* s, const svg_params* p, const uin
   if ((st = svg_qknorm_rope_layout(s, p, SVG_LAYOUT, qn, kn, v, nullptr, nullptr, nullptr, kinds, qp, kp, vp,
                                    stream)) != SVG_OK)
     return st;
+  if (!op)   // attention writes the model-order output directly (inverse layout in its epilogue)
+    return svg_block_sparse_attn_model_order(s, p, qp, kp, vp, kinds, row_ptr, col, full, out, nullptr, stream);
   if ((st = svg_block_sparse_attn(s, p, qp, kp, vp, kinds, row_ptr, col, full, op, nullptr, stream)) != SVG_OK)
     return st;
   return svg_inverse_layout(s, kinds, op, out, stream);

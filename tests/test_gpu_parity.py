@@ -215,14 +215,17 @@ def test_profile_bad_sample_index_reported():
 
 # --------------------------------------------------------------- attention
 
-def run_sparse(wl, qn, kn, v, kinds, want_lse=False):
+def run_sparse(wl, qn, kn, v, kinds, want_lse=False, model_order=False):
+    """Layout, block index and attention; the output comes back in model
+    order either through the inverse-layout pass or (model_order=True) from
+    the attention epilogue.  LSE is in the head's layout unless model_order."""
     pb = pb_of(wl)
     kd = dev(kinds)
     qp, kp, vp = svg.layout(pb, dev(qn), dev(kn), dev(v), kd)
     row_ptr, col, full = svg.build_block_index(pb, kd)
-    res = svg.block_sparse_attn(pb, qp, kp, vp, kd, row_ptr, col, full, want_lse=want_lse)
+    res = svg.block_sparse_attn(pb, qp, kp, vp, kd, row_ptr, col, full, want_lse=want_lse, model_order=model_order)
     op, lse = res if want_lse else (res, None)
-    out = svg.inverse_layout(pb, kd, op)
+    out = op if model_order else svg.inverse_layout(pb, kd, op)
     svg.sync_status()
     return out, lse
 
@@ -247,6 +250,23 @@ def test_attention_parity(key, kinds_mode):
     assert np.abs(lse_h[bh, pos] - ref_lse).max() < 5e-3
 
 
+@pytest.mark.parametrize("key", ["cfg0", "ragged128", "smallS128", "cfg2"])
+def test_attention_model_order_equals_inverse_layout_pass(key):
+    """The inverse layout fused into the attention epilogue stores exactly
+    the bits the separate pass produces, and the LSE at the same positions."""
+    wl, inp, qn, kn = case(key)
+    sh = oracle.shape_of(wl)
+    kinds = mixed_kinds(wl.H)
+    out_a, lse_a = run_sparse(wl, qn, kn, inp["v"], kinds, want_lse=True)
+    out_b, lse_b = run_sparse(wl, qn, kn, inp["v"], kinds, want_lse=True, model_order=True)
+    assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
+    lse_a = lse_a.cpu().numpy().reshape(wl.B * wl.H, wl.L)
+    lse_b = lse_b.cpu().numpy().reshape(wl.B * wl.H, wl.L)
+    for bh in range(wl.B * wl.H):
+        pos = np.array([oracle.perm(sh, int(kinds[bh]), t) for t in range(wl.L)])
+        assert np.array_equal(lse_b[bh], lse_a[bh, pos])
+
+
 def test_attention_dense_kinds_equal_dense_attention():
     wl, inp, qn, kn = case("smallS")
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
@@ -261,7 +281,7 @@ def test_attention_cfg3_sampled_rows():
     wl, inp, qn, kn = case("cfg3")
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
     kinds = np.array([W.SPATIAL if c == "S" else W.TEMPORAL for c in wl.planted], np.uint8)
-    out, _ = run_sparse(wl, qn, kn, inp["v"], kinds)
+    out, _ = run_sparse(wl, qn, kn, inp["v"], kinds, model_order=True)     # the launch bench.py times
     rows = rows_for("cfg3", wl)
     ref = oracle.attention_rows(sh, pr, kinds, qn, kn, inp["v"], rows)
     assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, "cfg3")
@@ -269,12 +289,13 @@ def test_attention_cfg3_sampled_rows():
 
 # ---------------------------------------------------------------- full step
 
-@pytest.mark.parametrize("key", ["cfg0", "smallS", "cfg1", "cfg2"])
-def test_full_step_end_to_end(key):
+@pytest.mark.parametrize("key,head_layout_out", [("cfg0", False), ("smallS", False), ("cfg1", False),
+                                                  ("cfg2", False), ("cfg0", True), ("cfg2", True)])
+def test_full_step_end_to_end(key, head_layout_out):
     wl, inp, qn, kn = case(key)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
     pb = pb_of(wl)
-    buf = svg.StepBuffers(pb, wl.n_samples)
+    buf = svg.StepBuffers(pb, wl.n_samples, head_layout_out=head_layout_out)
     out = svg.attention_step(pb, dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["gamma_q"]),
                              dev(inp["gamma_k"]), dev(inp["sample_idx"]), buf)
     svg.sync_status()
