@@ -47,6 +47,20 @@ def peaks():
     return dict(FALLBACK), "fallback"
 
 
+def reduce_over_ranks(times, work, device="cpu"):
+    """Max over ranks of `times`, sum over ranks of `work` (lists of floats);
+    the identity when no process group of more than one rank is up.  Every
+    rank must call it, in the same order."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(times, dtype=torch.float64, device=device)
+    w = torch.tensor(work, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.cpu()], [float(x) for x in w.cpu()]
+
+
 def kept_tile_flops(row_ptr: np.ndarray, col: np.ndarray, wl) -> float:
     """4*d*rows*cols summed over the listed (q-block, k-block) tiles."""
     nqb = wl.nqb
@@ -270,13 +284,11 @@ def run_gpu(args, rank, world, local_rank):
         del out_d, rp_d, col_d, full_d
     svg.sync_status()
 
-    # ---- max over ranks
-    vals = torch.tensor([total_ms, e2e_ms, stage_ms["attention"]], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms, attn_ms_max = (float(x) for x in vals.cpu())
+    # ---- times: max over ranks; work: sum over ranks (each rank runs its own layer)
+    (total_ms, e2e_ms, attn_ms_max), (flops_all,) = reduce_over_ranks(
+        [total_ms, e2e_ms, stage_ms["attention"]], [flops], device)
     ms_per_step = total_ms / args.steps
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = flops_all / (ms_per_step * 1e-3) / 1e12
     if rank != 0:
         return None
 
@@ -333,7 +345,7 @@ def run_gpu(args, rank, world, local_rank):
             "ms": round(dense_ms, 3), "tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 2),
             "speedup_sparse_attn_vs_dense": round(dense_ms / stage_ms["attention"], 3),
             "theoretical_speedup_tiles": round(dense_flops / flops, 3)},
-        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        "e2e": {"value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
