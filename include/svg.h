@@ -232,6 +232,24 @@ svg_status svg_sample_queries(uint64_t seed, int64_t Lv, int n, int32_t* host_ou
 size_t svg_rope_table_size(const svg_shape* shape, const svg_params* params);
 svg_status svg_rope_table_fill(const svg_shape* shape, const svg_params* params, float* host_out);
 
+/* What one layer's attention does at denoising step `step` of `total_steps`
+ * ("Sparse VideoGen" WeChat article, "其他优化方法": the first 25% of the
+ * generation steps run dense attention, the other 75% sparse; "Online Profiling
+ * Strategy": the best pattern changes from step to step, so it is profiled
+ * online).  *mode_out is
+ *   SVG_STEP_DENSE   if step < dense_fraction * total_steps (all heads DENSE;
+ *                    pass head_kind_in = all SVG_HEAD_DENSE to svg_attention_step),
+ *   SVG_STEP_PROFILE on the first sparse step and then every `reprofile_every`
+ *                    sparse steps (head_kind_in = NULL: profile, use the result),
+ *   SVG_STEP_REUSE   otherwise (head_kind_in = the last profiled kinds).
+ * reprofile_every = 1 profiles every sparse step, as the pages do; larger values
+ * are this library's option, not the pages'.
+ * SVG_ERR_INVALID_ARG for step outside [0, total_steps), total_steps < 1,
+ * dense_fraction outside [0, 1] or reprofile_every < 1.  Host only. */
+typedef enum { SVG_STEP_DENSE = 0, SVG_STEP_PROFILE = 1, SVG_STEP_REUSE = 2 } svg_step_mode;
+svg_status svg_step_policy(int step, int total_steps, float dense_fraction, int reprofile_every,
+                           int* mode_out);
+
 /* Entries that always suffice for svg_build_block_index: B*H*nqb*nkb. */
 int64_t svg_block_index_capacity(const svg_shape* shape, const svg_params* params);
 

@@ -10,6 +10,7 @@ from .build import LIB_PATH
 SVG_OK, SVG_ERR_INVALID_ARG, SVG_ERR_SHAPE, SVG_ERR_UNSUPPORTED = 0, 1, 2, 3
 SVG_ERR_ALIGNMENT, SVG_ERR_CAPACITY, SVG_ERR_CUDA, SVG_ERR_TIMEOUT = 4, 5, 6, 7
 SVG_HEAD_SPATIAL, SVG_HEAD_TEMPORAL, SVG_HEAD_DENSE = 0, 1, 2
+SVG_STEP_DENSE, SVG_STEP_PROFILE, SVG_STEP_REUSE = 0, 1, 2
 SVG_NORM_ROPE, SVG_LAYOUT = 1, 2
 
 
@@ -49,6 +50,7 @@ SIGNATURES = {
                                   _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
                                   _vp, _sz, _vp]),
     "svg_sample_queries": (_i32, [ctypes.c_uint64, _i64, _i32, _vp]),
+    "svg_step_policy": (_i32, [_i32, _i32, ctypes.c_float, _i32, ctypes.POINTER(ctypes.c_int)]),
     "svg_rope_table_size": (_sz, [_SP, _PP]),
     "svg_rope_table_fill": (_i32, [_SP, _PP, _vp]),
     "svg_block_index_capacity": (_i64, [_SP, _PP]),

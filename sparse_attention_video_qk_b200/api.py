@@ -281,3 +281,53 @@ def sparse_attention(pb: Problem, q_host, k_host, v_host, gamma_q, gamma_k, samp
             out_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
         out_host.copy_(o, non_blocking=True)
     return out_host
+
+
+# ------------------------------------------------------ denoising schedule --
+
+STEP_DENSE, STEP_PROFILE, STEP_REUSE = C.SVG_STEP_DENSE, C.SVG_STEP_PROFILE, C.SVG_STEP_REUSE
+
+
+def step_policy(step: int, total_steps: int, dense_fraction: float = 0.25, reprofile_every: int = 1) -> int:
+    """STEP_DENSE, STEP_PROFILE or STEP_REUSE for one layer at a denoising step
+    (svg_step_policy)."""
+    mode = ctypes.c_int(-1)
+    check(lib().svg_step_policy(int(step), int(total_steps), float(dense_fraction), int(reprofile_every),
+                                ctypes.byref(mode)), "svg_step_policy")
+    return mode.value
+
+
+class SparseAttentionLayer:
+    """One attention layer over a denoising schedule: all heads dense for the
+    first `dense_fraction` of the steps, then sparse with online profiling;
+    with reprofile_every > 1 the profiled head kinds are reused in between.
+    Each call runs the whole step through svg_attention_step."""
+
+    def __init__(self, pb: Problem, n_samples: int, total_steps: int, dense_fraction: float = 0.25,
+                 reprofile_every: int = 1, device="cuda"):
+        self.pb = pb
+        self.total_steps = total_steps
+        self.dense_fraction = dense_fraction
+        self.reprofile_every = reprofile_every
+        self.buffers = StepBuffers(pb, n_samples, device)
+        self.dense_kinds = torch.full((pb.B * pb.H,), DENSE, dtype=torch.uint8, device=device)
+        self.kinds = None          # the last profiled head kinds (device)
+        self.last_mode = None
+
+    def __call__(self, step: int, q, k, v, gamma_q, gamma_k, sample_idx, stream=None):
+        mode = step_policy(step, self.total_steps, self.dense_fraction, self.reprofile_every)
+        if mode == STEP_DENSE:
+            kinds_in = self.dense_kinds
+        elif mode == STEP_PROFILE:
+            kinds_in = None
+        else:
+            if self.kinds is None:
+                raise RuntimeError("REUSE step before any profiled step")
+            kinds_in = self.kinds
+        out = attention_step(self.pb, q, k, v, gamma_q, gamma_k, sample_idx, self.buffers, kinds_in=kinds_in,
+                             stream=stream)
+        if mode == STEP_PROFILE:
+            self.kinds = self.buffers.kinds.clone()
+        self.last_mode = mode
+        return out
+

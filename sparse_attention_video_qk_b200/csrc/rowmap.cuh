@@ -87,6 +87,8 @@ struct RowmapArgs {
   float eps;
   int split0, split1;        // widths of the t and h sections (w = d - split0 - split1)
   int rope_off1, rope_off2;  // table offsets (in float2) of the h and w sections
+  int rope_vec;              // 1: every section is a multiple of 8 wide, so a lane's 4 pairs share a
+                             //    section and sit next to each other in the table
   FastDiv divF, divS, divWs;
 };
 
@@ -194,14 +196,30 @@ __global__ void __launch_bounds__(256, kRowmapBlocksPerSM) rowmap_kernel(const R
           if (tok[u] < g.Lv) {
             const int f = fdiv(tok[u], a.divS), s = tok[u] - f * g.S;
             const int yy = fdiv(s, a.divWs), xx = s - yy * g.Ws;
+            float2 cs[4];
+            if (STAGED && a.rope_vec) {
+              // the lane's 4 (cos, sin) pairs in two 16-byte shared-memory loads
+              const int pos = sec[0] == 0 ? f : (sec[0] == 1 ? yy : xx);
+              const float4* t4 = reinterpret_cast<const float4*>(rope_s + tab[0] + pos * stride[0]);
+              const float4 c01 = t4[0], c23 = t4[1];
+              cs[0] = make_float2(c01.x, c01.y);
+              cs[1] = make_float2(c01.z, c01.w);
+              cs[2] = make_float2(c23.x, c23.y);
+              cs[3] = make_float2(c23.z, c23.w);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 4; i++) {
+                const int pos = sec[i] == 0 ? f : (sec[i] == 1 ? yy : xx);
+                cs[i] = STAGED ? rope_s[tab[i] + pos * stride[i]] : __ldg(a.rope + tab[i] + pos * stride[i]);
+              }
+            }
 #pragma unroll
             for (int i = 0; i < 4; i++) {
-              const int pos = sec[i] == 0 ? f : (sec[i] == 1 ? yy : xx);
-              const float2 cs = STAGED ? rope_s[tab[i] + pos * stride[i]] : __ldg(a.rope + tab[i] + pos * stride[i]);
               // (u, v) -> (u c - v s, u s + v c) = (u, u) * (c, s) + (-v, v) * (s, c)
               float u0, u1;
               unpack_f2(v2[i], u0, u1);
-              v2[i] = fma_f2(pack_f2(-u1, u1), pack_f2(cs.y, cs.x), mul_f2(pack_f2(u0, u0), pack_f2(cs.x, cs.y)));
+              v2[i] = fma_f2(pack_f2(-u1, u1), pack_f2(cs[i].y, cs[i].x),
+                             mul_f2(pack_f2(u0, u0), pack_f2(cs[i].x, cs[i].y)));
             }
           }
           float r[8];

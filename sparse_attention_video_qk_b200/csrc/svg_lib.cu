@@ -219,6 +219,21 @@ const char* svg_status_string(svg_status s) {
   return "unknown status";
 }
 
+svg_status svg_step_policy(int step, int total_steps, float dense_fraction, int reprofile_every, int* mode_out) {
+  if (!mode_out || total_steps < 1 || step < 0 || step >= total_steps || !(dense_fraction >= 0.f) ||
+      !(dense_fraction <= 1.f) || reprofile_every < 1)
+    return SVG_ERR_INVALID_ARG;
+  // dense iff step / total_steps < dense_fraction, decided in double
+  const double cut = static_cast<double>(dense_fraction) * total_steps;
+  if (static_cast<double>(step) < cut) {
+    *mode_out = SVG_STEP_DENSE;
+    return SVG_OK;
+  }
+  const int first_sparse = static_cast<int>(std::ceil(cut));
+  *mode_out = ((step - first_sparse) % reprofile_every == 0) ? SVG_STEP_PROFILE : SVG_STEP_REUSE;
+  return SVG_OK;
+}
+
 svg_status svg_sample_queries(uint64_t seed, int64_t Lv, int n, int32_t* host_out) {
   if (!host_out || n <= 0 || Lv <= 0 || n > Lv || Lv > INT32_MAX) return SVG_ERR_INVALID_ARG;
   // partial Fisher-Yates over 0..Lv-1; only the touched slots are remembered
@@ -350,6 +365,7 @@ svg_status svg_qknorm_rope_layout(const svg_shape* s, const svg_params* p, int f
   a.split1 = p->rope_split[1];
   a.rope_off1 = s->F * (p->rope_split[0] / 2);
   a.rope_off2 = a.rope_off1 + s->Hs * (p->rope_split[1] / 2);
+  a.rope_vec = (p->rope_split[0] % 8 == 0 && p->rope_split[1] % 8 == 0 && p->rope_split[2] % 8 == 0) ? 1 : 0;
   return launch_rowmap(a, s->d, static_cast<cudaStream_t>(stream));
 }
 

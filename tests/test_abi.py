@@ -127,3 +127,18 @@ def test_noalloc_capacity_limit(L):
                                            None) == C.SVG_ERR_CAPACITY
         assert L.svg_profile_heads_noalloc(ctypes.byref(sh), ctypes.byref(pr), p, p, p, p, 65, None, p,
                                            None) == C.SVG_ERR_INVALID_ARG
+
+
+def test_step_policy_schedule(L):
+    """First 25% of the steps dense, then profiling every sparse step (or every
+    `reprofile_every` sparse steps, reusing the kinds in between)."""
+    D, P, R = api.STEP_DENSE, api.STEP_PROFILE, api.STEP_REUSE
+    assert [api.step_policy(t, 50) for t in range(50)] == [D] * 13 + [P] * 37   # t < 12.5
+    assert [api.step_policy(t, 8) for t in range(8)] == [D, D, P, P, P, P, P, P]
+    assert [api.step_policy(t, 8, 0.25, 3) for t in range(8)] == [D, D, P, R, R, P, R, R]
+    assert [api.step_policy(t, 4, 0.0) for t in range(4)] == [P] * 4
+    assert [api.step_policy(t, 4, 1.0) for t in range(4)] == [D] * 4
+    for bad in [(-1, 4, 0.25, 1), (4, 4, 0.25, 1), (0, 0, 0.25, 1), (0, 4, 1.5, 1), (0, 4, -0.1, 1),
+                (0, 4, float("nan"), 1), (0, 4, 0.25, 0)]:
+        with pytest.raises(C.SVGError):
+            api.step_policy(*bad)

@@ -53,8 +53,11 @@ CASES = {
     "oneframe": W.small_workload(d=128, H=2, F=1, Hs=12, Ws=20, T=7, w=0, r=30, n_samples=8),
     # wide windows that reduce to dense
     "wide": W.small_workload(d=64, H=2, F=5, Hs=6, Ws=7, T=9, w=4, r=41, n_samples=8),
+    # RoPE sections not multiples of 8 wide: a lane's 4 pairs straddle two sections
+    "oddsplit": W.small_workload(d=64, H=2, F=4, Hs=5, Ws=6, T=3, w=1, r=4, n_samples=8, rope_split=(18, 22, 24)),
 }
-FULL_ROW_CASES = ("cfg0", "ragged128", "tiny64", "smallS", "smallS128", "smallS_T0", "oneframe", "wide")
+FULL_ROW_CASES = ("cfg0", "ragged128", "tiny64", "smallS", "smallS128", "smallS_T0", "oneframe", "wide",
+                  "oddsplit")
 
 
 def pb_of(wl):
@@ -75,7 +78,7 @@ def rows_for(key, wl):
 
 # ------------------------------------------------------------ QK-Norm + RoPE
 
-@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "ragged128", "tiny64", "oneframe"])
+@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "ragged128", "tiny64", "oneframe", "oddsplit"])
 def test_qknorm_rope_within_one_ulp(key):
     wl, inp, qn_ref, kn_ref = case(key)
     pb = pb_of(wl)
@@ -318,3 +321,23 @@ def test_host_buffer_api_matches_device_api():
                                dev(inp["gamma_k"]), dev(inp["sample_idx"]), buf)
     svg.sync_status()
     assert torch.equal(out_h.view(torch.int16), out_d.cpu().view(torch.int16))
+
+
+def test_layer_schedule_dense_then_profiled_then_reused():
+    """SparseAttentionLayer over 4 denoising steps: step 0 dense, step 1
+    profiled, step 2 reuses step 1's kinds, step 3 profiles again."""
+    wl, inp, qn, kn = case("cfg0")
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    layer = svg.SparseAttentionLayer(pb_of(wl), wl.n_samples, total_steps=4, dense_fraction=0.25, reprofile_every=2)
+    args = tuple(dev(inp[k]) for k in ("q", "k", "v", "gamma_q", "gamma_k", "sample_idx"))
+    _, kinds_ref = oracle.profile(sh, pr, qn, kn, inp["v"], inp["sample_idx"])
+    rows = rows_for("cfg0", wl)
+    modes = [svg.STEP_DENSE, svg.STEP_PROFILE, svg.STEP_REUSE, svg.STEP_PROFILE]
+    for t in range(4):
+        out = layer(t, *args)
+        svg.sync_status()
+        assert layer.last_mode == modes[t]
+        kinds = np.full(wl.H, W.DENSE, np.uint8) if t == 0 else kinds_ref
+        ref = oracle.attention_rows(sh, pr, kinds, qn, kn, inp["v"], rows)
+        assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, f"step {t}")
+    assert np.array_equal(layer.kinds.cpu().numpy(), kinds_ref)
