@@ -189,17 +189,21 @@ def run_gpu(args, rank, world, local_rank):
         """The step as its five C-ABI calls (the same calls svg_attention_step makes)."""
         b = buf
         return [
-            ("qknorm_rope", lambda: lib.svg_qknorm_rope_layout(ctypes.byref(sh), ctypes.byref(pr), 1, P(q), P(k), None,
-                                                              P(gq), P(gk), P(b.table), None, P(b.qn), P(b.kn), None,
-                                                              cs)),
-            ("profile", lambda: lib.svg_profile_heads(ctypes.byref(sh), ctypes.byref(pr), P(b.qn), P(b.kn), P(v),
-                                                      P(si), int(si.numel()), P(b.workspace), b.workspace.numel(),
-                                                      P(b.mse), P(b.kinds), cs)),
+            # 1. QK-Norm + RoPE of K
+            ("k_norm_rope", lambda: lib.svg_qknorm_rope_layout(ctypes.byref(sh), ctypes.byref(pr), 1, None, P(k),
+                                                              None, None, P(gk), P(b.table), None, None, P(b.kn),
+                                                              None, cs)),
+            # 2. profiling from raw Q (sampled rows normalised in the kernel)
+            ("profile", lambda: lib.svg_profile_heads_raw_q(ctypes.byref(sh), ctypes.byref(pr), P(q), P(gq),
+                                                            P(b.table), P(b.kn), P(v), P(si), int(si.numel()),
+                                                            P(b.workspace), b.workspace.numel(), P(b.mse),
+                                                            P(b.kinds), cs)),
             ("block_index", lambda: lib.svg_build_block_index(ctypes.byref(sh), ctypes.byref(pr), P(b.kinds),
                                                               P(b.row_ptr), P(b.col), P(b.full), b.capacity, cs)),
-            ("layout", lambda: lib.svg_qknorm_rope_layout(ctypes.byref(sh), ctypes.byref(pr), 2, P(b.qn), P(b.kn),
-                                                          P(v), None, None, None, P(b.kinds), P(b.qp), P(b.kp),
-                                                          P(b.vp), cs)),
+            # 4. QK-Norm + RoPE of Q and the layout transform of Q, K, V in one pass
+            ("q_norm_rope_layout", lambda: lib.svg_qknorm_rope_layout(
+                ctypes.byref(sh), ctypes.byref(pr), 3, P(q), P(b.kn), P(v), P(gq), None, P(b.table), P(b.kinds),
+                P(b.qp), P(b.kp), P(b.vp), cs)),
             # attention with the inverse layout in its epilogue: writes `out` in model order
             ("attention", lambda: lib.svg_block_sparse_attn_model_order(
                 ctypes.byref(sh), ctypes.byref(pr), P(b.qp), P(b.kp), P(b.vp), P(b.kinds), P(b.row_ptr),
@@ -299,7 +303,7 @@ def run_gpu(args, rank, world, local_rank):
                            else ("attention.cuh", f"attn_kernel<{wl.d}>"))
     traffic = traffic_from_profile(attn_src, "attention_hunyuan_cfg3.md") if args.config == 3 else None
     d, L, BH = wl.d, wl.L, wl.B * wl.H
-    stage_bytes = {"qknorm_rope": 8.0 * BH * L * d, "layout": 12.0 * BH * L * d,
+    stage_bytes = {"k_norm_rope": 4.0 * BH * L * d, "q_norm_rope_layout": 12.0 * BH * L * d,
                    "profile": 4.0 * BH * L * d}
     line = {
         "metric": METRIC,

@@ -90,9 +90,14 @@ enum { SVG_NORM_ROPE = 1, SVG_LAYOUT = 2 };
  *     head_kind is TEMPORAL, video row f*S+s goes to s*F+f (S = Hs*Ws); text rows and
  *     other heads stay in place.  v (required with LAYOUT) is moved the same way
  *     without normalisation.
- * q, k, v, q_out, k_out, v_out: device bf16 [B,H,L,d].  v/v_out are used only with
- *   SVG_LAYOUT (may be NULL otherwise).
- * gamma_q, gamma_k: device fp32 [d]; required with SVG_NORM_ROPE.
+ * q, k, v, q_out, k_out, v_out: device bf16 [B,H,L,d].  Each tensor comes with its
+ *   output or is NULL with it (q or k must be given); v is given only with SVG_LAYOUT,
+ *   which requires it.
+ * gamma_q, gamma_k: device fp32 [d].  With SVG_NORM_ROPE, q (k) is normalised iff
+ *   gamma_q (gamma_k) is given; at least one must be.  With SVG_LAYOUT a tensor
+ *   without its gamma is only moved, so {q raw, k already normalised, v} with only
+ *   gamma_q gives the step's single fused pass; without SVG_LAYOUT every given
+ *   tensor must be normalised (e.g. k alone).
  * rope_table: device fp32 table of svg_rope_table_size() floats written on the host
  *   by svg_rope_table_fill() and copied by the caller; required with SVG_NORM_ROPE.
  * head_kind: device uint8 [B*H]; required with SVG_LAYOUT. */
@@ -118,6 +123,19 @@ svg_status svg_profile_heads(const svg_shape* shape, const svg_params* params,
                              const uint16_t* qn, const uint16_t* kn, const uint16_t* v,
                              const int32_t* sample_idx, int n, void* workspace, size_t workspace_bytes,
                              float* mse_out, uint8_t* head_kind_out, void* stream);
+
+/* Stage 2 on raw Q: as svg_profile_heads, but q is the un-normalised Q (model order)
+ * and each sampled row gets QK-Norm + RoPE inside the kernel, with the same device
+ * routine (same lane split and operation order) as svg_qknorm_rope_layout, so the
+ * rows are bit-identical to that stage's output.  This lets a step normalise Q in
+ * the same pass that moves it into the heads' layouts.
+ * gamma_q: device fp32 [d]; rope_table: as for svg_qknorm_rope_layout; kn: K after
+ * QK-Norm + RoPE.  Other arguments and errors as for svg_profile_heads. */
+svg_status svg_profile_heads_raw_q(const svg_shape* shape, const svg_params* params,
+                                   const uint16_t* q, const float* gamma_q, const float* rope_table,
+                                   const uint16_t* kn, const uint16_t* v,
+                                   const int32_t* sample_idx, int n, void* workspace, size_t workspace_bytes,
+                                   float* mse_out, uint8_t* head_kind_out, void* stream);
 
 /* Stage 2 without a caller-provided workspace.  The paper has no counterpart:
  * this entry point exists for callers that can hand the library only their
@@ -199,13 +217,21 @@ svg_status svg_block_sparse_attn_model_order(const svg_shape* shape, const svg_p
 svg_status svg_inverse_layout(const svg_shape* shape, const uint8_t* head_kind,
                               const uint16_t* src, uint16_t* dst, void* stream);
 
-/* The five stages in order on one stream (profiling skipped when
- * head_kind_in != NULL, whose kinds are then used).  All buffers are device
- * memory owned by the caller:
- *   qn, kn, qp, kp, vp: bf16 [B,H,L,d] intermediates;
- *   op: bf16 [B,H,L,d] attention output in the head's layout, or NULL -- with
- *   NULL, the attention writes `out` in model order directly
- *   (svg_block_sparse_attn_model_order) and no inverse pass runs;
+/* The whole step on one stream, in five passes:
+ *   1. QK-Norm + RoPE of K into kn (frame-major);
+ *   2. profiling (svg_profile_heads_raw_q: the sampled Q rows are normalised in
+ *      the kernel) -- skipped when head_kind_in != NULL, whose kinds are used;
+ *   3. the block index;
+ *   4. one pass that normalises Q and writes Q, kn and V in the heads' layouts
+ *      (qp, kp, vp);
+ *   5. block-sparse attention; with op = NULL it writes `out` in model order
+ *      directly (svg_block_sparse_attn_model_order), otherwise it writes op in the
+ *      heads' layout and svg_inverse_layout produces `out`.
+ * Every output equals running the stages one by one with svg_qknorm_rope_layout
+ * (NORM_ROPE), svg_profile_heads, svg_build_block_index, svg_qknorm_rope_layout
+ * (LAYOUT) and svg_block_sparse_attn + svg_inverse_layout: the norm routine is
+ * the same in every pass.  All buffers are device memory owned by the caller:
+ *   kn, qp, kp, vp: bf16 [B,H,L,d] intermediates; op: bf16 [B,H,L,d] or NULL;
  *   out: bf16 [B,H,L,d] final output in model order;
  *   head_kind_out: uint8 [B*H]; mse_out: fp32 [B*H*2] or NULL;
  *   row_ptr/col/full: block index with `capacity` entries;
@@ -214,7 +240,7 @@ svg_status svg_attention_step(const svg_shape* shape, const svg_params* params,
                               const uint16_t* q, const uint16_t* k, const uint16_t* v,
                               const float* gamma_q, const float* gamma_k, const float* rope_table,
                               const int32_t* sample_idx, int n, const uint8_t* head_kind_in,
-                              uint16_t* qn, uint16_t* kn, uint16_t* qp, uint16_t* kp, uint16_t* vp,
+                              uint16_t* kn, uint16_t* qp, uint16_t* kp, uint16_t* vp,
                               uint16_t* op, uint16_t* out, uint8_t* head_kind_out, float* mse_out,
                               int32_t* row_ptr, int32_t* col, uint8_t* full, int64_t capacity,
                               void* workspace, size_t workspace_bytes, void* stream);

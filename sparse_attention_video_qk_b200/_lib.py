@@ -41,13 +41,14 @@ _SP, _PP = ctypes.POINTER(SvgShape), ctypes.POINTER(SvgParams)
 SIGNATURES = {
     "svg_qknorm_rope_layout": (_i32, [_SP, _PP, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "svg_profile_heads": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp, _vp, _vp]),
+    "svg_profile_heads_raw_q": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _sz, _vp, _vp, _vp]),
     "svg_profile_heads_noalloc": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp]),
     "svg_build_block_index": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _i64, _vp]),
     "svg_block_sparse_attn": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "svg_block_sparse_attn_model_order": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "svg_inverse_layout": (_i32, [_SP, _vp, _vp, _vp, _vp]),
     "svg_attention_step": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
-                                  _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
+                                  _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
                                   _vp, _sz, _vp]),
     "svg_sample_queries": (_i32, [ctypes.c_uint64, _i64, _i32, _vp]),
     "svg_step_policy": (_i32, [_i32, _i32, ctypes.c_float, _i32, ctypes.POINTER(ctypes.c_int)]),

@@ -126,7 +126,8 @@ def qknorm_rope_layout(pb: Problem, q, k, v=None, gamma_q=None, gamma_k=None, ta
     Returns (q_out, k_out, v_out or None)."""
     sh, pr = pb.c_shape(), pb.c_params()
     if out is None:
-        out = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v) if (flags & C.SVG_LAYOUT) else None)
+        like = lambda t: torch.empty_like(t) if t is not None else None
+        out = (like(q), like(k), like(v) if (flags & C.SVG_LAYOUT) else None)
     qo, ko, vo = out
     st = lib().svg_qknorm_rope_layout(ctypes.byref(sh), ctypes.byref(pr), flags, _p(q), _p(k), _p(v),
                                       _p(gamma_q), _p(gamma_k), _p(table), _p(kinds), _p(qo), _p(ko), _p(vo),
@@ -160,6 +161,26 @@ def profile_heads(pb: Problem, qn, kn, v, sample_idx, workspace=None, kinds_out=
                                  _p(workspace), workspace.numel() * workspace.element_size(), _p(mse_out),
                                  _p(kinds_out), _stream(stream))
     check(st, "svg_profile_heads")
+    return kinds_out, mse_out
+
+
+def profile_heads_raw_q(pb: Problem, q, gamma_q, table, kn, v, sample_idx, workspace=None, kinds_out=None,
+                        mse_out=None, stream=None):
+    """svg_profile_heads_raw_q: profiling from raw Q (the sampled rows are
+    normalised in the kernel).  Returns (kinds uint8 [B*H], mse fp32 [B*H, 2])."""
+    sh, pr = pb.c_shape(), pb.c_params()
+    n = int(sample_idx.numel())
+    if workspace is None:
+        workspace = torch.empty(profile_workspace_size(pb, n), dtype=torch.uint8, device=q.device)
+    if kinds_out is None:
+        kinds_out = torch.empty(pb.B * pb.H, dtype=torch.uint8, device=q.device)
+    if mse_out is None:
+        mse_out = torch.empty(pb.B * pb.H, 2, dtype=torch.float32, device=q.device)
+    st = lib().svg_profile_heads_raw_q(ctypes.byref(sh), ctypes.byref(pr), _p(q), _p(gamma_q), _p(table), _p(kn),
+                                       _p(v), _p(sample_idx), n, _p(workspace),
+                                       workspace.numel() * workspace.element_size(), _p(mse_out), _p(kinds_out),
+                                       _stream(stream))
+    check(st, "svg_profile_heads_raw_q")
     return kinds_out, mse_out
 
 
@@ -233,7 +254,7 @@ class StepBuffers:
         mk = lambda: torch.empty(shp, dtype=torch.bfloat16, device=device)
         self.pb = pb
         self.n = n_samples
-        self.qn, self.kn, self.qp, self.kp, self.vp, self.out = (mk() for _ in range(6))
+        self.kn, self.qp, self.kp, self.vp, self.out = (mk() for _ in range(5))
         self.op = mk() if head_layout_out else None
         self.kinds = torch.empty(pb.B * pb.H, dtype=torch.uint8, device=device)
         self.mse = torch.empty(pb.B * pb.H, 2, dtype=torch.float32, device=device)
@@ -254,7 +275,7 @@ def attention_step(pb: Problem, q, k, v, gamma_q, gamma_k, sample_idx, buffers: 
     sh, pr = pb.c_shape(), pb.c_params()
     st = lib().svg_attention_step(
         ctypes.byref(sh), ctypes.byref(pr), _p(q), _p(k), _p(v), _p(gamma_q), _p(gamma_k), _p(b.table),
-        _p(sample_idx), int(sample_idx.numel()), _p(kinds_in), _p(b.qn), _p(b.kn), _p(b.qp), _p(b.kp), _p(b.vp),
+        _p(sample_idx), int(sample_idx.numel()), _p(kinds_in), _p(b.kn), _p(b.qp), _p(b.kp), _p(b.vp),
         _p(b.op), _p(b.out), _p(b.kinds), _p(b.mse), _p(b.row_ptr), _p(b.col), _p(b.full), b.capacity,
         _p(b.workspace), b.workspace.numel(), _stream(stream))
     check(st, "svg_attention_step")

@@ -24,6 +24,7 @@
 #pragma once
 
 #include "attention.cuh"
+#include "norm_rope.cuh"
 #include "svg_common.cuh"
 
 namespace svg {
@@ -55,7 +56,9 @@ __host__ __device__ inline size_t prof_workspace_bytes(int BH, int L, int D, int
 struct ProfArgs {
   Geometry g;
   float scale_log2;
-  const uint16_t* q;
+  const uint16_t* q;   // normalised Q, or raw Q when gamma_q is set
+  const float* gamma_q;  // non-null: the gathered rows get QK-Norm + RoPE here (norm_rope.cuh)
+  RopeArgs rope;
   const int32_t* sample;
   int n;
   int nchunk;
@@ -139,20 +142,33 @@ __global__ void __launch_bounds__(ProfCfg<D>::THREADS, 1)
   // Gather the sampled Q rows into both halves of the 128-row A operand, in
   // the 128-byte-swizzled K-major layout TMA would produce (16-byte chunk c of
   // row r stored at chunk c ^ (r % 8) of that row's 128-byte panel line).
+  // Consecutive lanes take consecutive chunks of one row, and every warp is
+  // either fully inside the loop or out of it (THREADS and 128*D/8 are
+  // multiples of 32), so the norm routine's butterfly sees whole rows.
   {
+    static_assert(C::THREADS % 32 == 0 && (128 * (D / 8)) % 32 == 0, "whole warps in the gather");
     const int64_t hoff = static_cast<int64_t>(bh) * g.L * D;
+    const bool norm = a.gamma_q != nullptr;
+    uint64_t gam[4] = {0ull, 0ull, 0ull, 0ull};
+    RopeLane rl{};
+    if (norm) {
+      load_gain(a.gamma_q, threadIdx.x % (D / 8), gam);
+      rl = rope_lane<D>(threadIdx.x % (D / 8), a.rope);
+    }
     for (int i = threadIdx.x; i < 128 * (D / 8); i += C::THREADS) {
       const int r = i / (D / 8), c = i % (D / 8);
       const int sr = r & 63;
       uint4 val = make_uint4(0, 0, 0, 0);
+      int tok = 0;
       if (sr < a.n) {
-        int tok = a.sample[sr];
+        tok = a.sample[sr];
         if (tok < 0 || tok >= g.L) {
           atomicOr(&g_error_word, kErrBadIndex);
           tok = 0;
         }
         val = __ldg(reinterpret_cast<const uint4*>(a.q + hoff + static_cast<int64_t>(tok) * D) + c);
       }
+      if (norm) val = norm_rope_vec<D, false>(val, tok, g, gam, rl, a.rope, a.rope.table);
       const int panel = c >> 3, cc = c & 7;
       *reinterpret_cast<uint4*>(sQ + panel * C::PANEL + r * 128 + ((cc ^ (r & 7)) << 4)) = val;
     }

@@ -127,10 +127,25 @@ bool set_smem(K kernel, int bytes) {
 
 // ------------------------------------------------------------- rowmap ----
 
+// RoPE table layout and constants of the norm routine (norm_rope.cuh).
+RopeArgs make_rope_args(const svg_shape* s, const svg_params* p, const float* rope_table) {
+  RopeArgs r{};
+  r.table = reinterpret_cast<const float2*>(rope_table);
+  r.eps = p ? p->eps : 0.f;
+  if (p) {
+    r.split0 = p->rope_split[0];
+    r.split1 = p->rope_split[1];
+    r.off1 = s->F * (p->rope_split[0] / 2);
+    r.off2 = r.off1 + s->Hs * (p->rope_split[1] / 2);
+    r.vec = (p->rope_split[0] % 8 == 0 && p->rope_split[1] % 8 == 0 && p->rope_split[2] % 8 == 0) ? 1 : 0;
+  }
+  r.divS = make_fastdiv(s->Hs * s->Ws);
+  r.divWs = make_fastdiv(s->Ws);
+  return r;
+}
+
 svg_status launch_rowmap(RowmapArgs a, int D, cudaStream_t st) {
   a.divF = make_fastdiv(a.g.F);
-  a.divS = make_fastdiv(a.g.S);
-  a.divWs = make_fastdiv(a.g.Ws);
   const int unit_rows = 8 * (32 / (D / 8)) * kRowmapSteps * kRowmapUnitSteps;
   const int64_t nunits = static_cast<int64_t>(a.ntensor) * a.g.BH * ((a.g.L + unit_rows - 1) / unit_rows);
   if (nunits > INT32_MAX) return SVG_ERR_UNSUPPORTED;
@@ -160,13 +175,18 @@ svg_status launch_rowmap(RowmapArgs a, int D, cudaStream_t st) {
 // Profiling: the tensor-core partial kernel over key chunks, the per-row
 // merge and the per-head choice.  `workspace` holds
 // prof_workspace_bytes(BH, L, d, max_chunks) bytes.
+// qn holds normalised Q, or raw Q when gamma_q is given (the sampled rows are
+// then normalised in the kernel with rope_table).
 svg_status launch_profile(const svg_shape* s, const svg_params* p, const uint16_t* qn, const uint16_t* kn,
                           const uint16_t* v, const int32_t* sample_idx, int n, void* workspace, int max_chunks,
-                          float* mse_out, uint8_t* head_kind_out, cudaStream_t cs) {
+                          float* mse_out, uint8_t* head_kind_out, cudaStream_t cs, const float* gamma_q = nullptr,
+                          const float* rope_table = nullptr) {
   ProfArgs a{};
   a.g = make_geometry(s, p);
   a.scale_log2 = scale_of(s, p) * 1.4426950408889634f;
   a.q = qn;
+  a.gamma_q = gamma_q;
+  a.rope = make_rope_args(s, p, rope_table);
   a.sample = sample_idx;
   a.n = n;
   const int ntiles = (a.g.L + kProfKeys - 1) / kProfKeys;
@@ -332,40 +352,42 @@ svg_status svg_qknorm_rope_layout(const svg_shape* s, const svg_params* p, int f
   if (!p) return SVG_ERR_INVALID_ARG;
   if ((st = check_params(s, p, false)) != SVG_OK) return st;
   if (flags == 0 || (flags & ~(SVG_NORM_ROPE | SVG_LAYOUT))) return SVG_ERR_INVALID_ARG;
-  if (!q || !k || !q_out || !k_out) return SVG_ERR_INVALID_ARG;
-  if (flags & SVG_NORM_ROPE) {
-    if (!gamma_q || !gamma_k || !rope_table) return SVG_ERR_INVALID_ARG;
+  const bool norm = (flags & SVG_NORM_ROPE) != 0, layout = (flags & SVG_LAYOUT) != 0;
+  // each tensor is given with its output or not at all
+  if (!q != !q_out || !k != !k_out || !v != !v_out || (!q && !k)) return SVG_ERR_INVALID_ARG;
+  const bool norm_q = norm && q && gamma_q, norm_k = norm && k && gamma_k;
+  if (norm) {
+    if (!(norm_q || norm_k) || !rope_table) return SVG_ERR_INVALID_ARG;
     if ((st = check_rope(s, p)) != SVG_OK) return st;
   }
-  if (flags & SVG_LAYOUT) {
-    if (!v || !v_out || !head_kind) return SVG_ERR_INVALID_ARG;
+  if (layout) {
+    if (!v || !head_kind) return SVG_ERR_INVALID_ARG;
+  } else if (v || (q && !norm_q) || (k && !norm_k)) {
+    return SVG_ERR_INVALID_ARG;       // without LAYOUT, every given tensor is normalised
   }
   const void* ptrs[] = {q, k, v, q_out, k_out, v_out, gamma_q, gamma_k, rope_table};
   for (const void* ptr : ptrs)
     if (ptr && !aligned16(ptr)) return SVG_ERR_ALIGNMENT;
-  if (q == q_out || k == k_out || (v && v == v_out)) return SVG_ERR_INVALID_ARG;
+  if ((q && q == q_out) || (k && k == k_out) || (v && v == v_out)) return SVG_ERR_INVALID_ARG;
   RowmapArgs a{};
   a.g = make_geometry(s, p);
-  a.flags = flags;
-  a.ntensor = (flags & SVG_LAYOUT) ? 3 : 2;
-  a.norm_tensors = (flags & SVG_NORM_ROPE) ? 2 : 0;
-  a.src[0] = q;
-  a.src[1] = k;
-  a.src[2] = v;
-  a.dst[0] = q_out;
-  a.dst[1] = k_out;
-  a.dst[2] = v_out;
-  a.gamma[0] = gamma_q;
-  a.gamma[1] = gamma_k;
-  a.rope = reinterpret_cast<const float2*>(rope_table);
-  a.rope_floats = (flags & SVG_NORM_ROPE) ? static_cast<int>(svg_rope_table_size(s, p)) : 0;
+  a.flags = flags & SVG_LAYOUT;
+  // normalised tensors first, then the ones that only move
+  auto add = [&](const uint16_t* src, uint16_t* dst, const float* gamma) {
+    a.src[a.ntensor] = src;
+    a.dst[a.ntensor] = dst;
+    a.gamma[a.ntensor] = gamma;
+    a.ntensor++;
+  };
+  if (norm_q) add(q, q_out, gamma_q);
+  if (norm_k) add(k, k_out, gamma_k);
+  a.norm_tensors = a.ntensor;
+  if (q && !norm_q) add(q, q_out, nullptr);
+  if (k && !norm_k) add(k, k_out, nullptr);
+  if (v) add(v, v_out, nullptr);
   a.kind = head_kind;
-  a.eps = p->eps;
-  a.split0 = p->rope_split[0];
-  a.split1 = p->rope_split[1];
-  a.rope_off1 = s->F * (p->rope_split[0] / 2);
-  a.rope_off2 = a.rope_off1 + s->Hs * (p->rope_split[1] / 2);
-  a.rope_vec = (p->rope_split[0] % 8 == 0 && p->rope_split[1] % 8 == 0 && p->rope_split[2] % 8 == 0) ? 1 : 0;
+  a.rope_floats = norm ? static_cast<int>(svg_rope_table_size(s, p)) : 0;
+  a.rope = make_rope_args(s, p, norm ? rope_table : nullptr);
   return launch_rowmap(a, s->d, static_cast<cudaStream_t>(stream));
 }
 
@@ -383,6 +405,7 @@ svg_status svg_inverse_layout(const svg_shape* s, const uint8_t* head_kind, cons
   a.src[0] = src;
   a.dst[0] = dst;
   a.kind = head_kind;
+  a.rope = make_rope_args(s, nullptr, nullptr);
   return launch_rowmap(a, s->d, static_cast<cudaStream_t>(stream));
 }
 
@@ -400,6 +423,25 @@ svg_status svg_profile_heads(const svg_shape* s, const svg_params* p, const uint
   if (workspace_bytes < svg_profile_workspace_size(s, n)) return SVG_ERR_CAPACITY;
   return launch_profile(s, p, qn, kn, v, sample_idx, n, workspace, prof_chunks(s->B * s->H, s->L), mse_out,
                         head_kind_out, static_cast<cudaStream_t>(stream));
+}
+
+svg_status svg_profile_heads_raw_q(const svg_shape* s, const svg_params* p, const uint16_t* q, const float* gamma_q,
+                                   const float* rope_table, const uint16_t* kn, const uint16_t* v,
+                                   const int32_t* sample_idx, int n, void* workspace, size_t workspace_bytes,
+                                   float* mse_out, uint8_t* head_kind_out, void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if ((st = check_params(s, p, false)) != SVG_OK) return st;
+  if ((st = check_rope(s, p)) != SVG_OK) return st;
+  if (!q || !gamma_q || !rope_table || !kn || !v || !sample_idx || !workspace || !head_kind_out)
+    return SVG_ERR_INVALID_ARG;
+  if (n < 1 || n > kProfRows) return SVG_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, gamma_q, rope_table, kn, v, workspace, mse_out};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return SVG_ERR_ALIGNMENT;
+  if (workspace_bytes < svg_profile_workspace_size(s, n)) return SVG_ERR_CAPACITY;
+  return launch_profile(s, p, q, kn, v, sample_idx, n, workspace, prof_chunks(s->B * s->H, s->L), mse_out,
+                        head_kind_out, static_cast<cudaStream_t>(stream), gamma_q, rope_table);
 }
 
 svg_status svg_build_block_index(const svg_shape* s, const svg_params* p, const uint8_t* head_kind,
@@ -488,27 +530,32 @@ svg_status svg_block_sparse_attn_model_order(const svg_shape* s, const svg_param
 
 svg_status svg_attention_step(const svg_shape* s, const svg_params* p, const uint16_t* q, const uint16_t* k,
                               const uint16_t* v, const float* gamma_q, const float* gamma_k, const float* rope_table,
-                              const int32_t* sample_idx, int n, const uint8_t* head_kind_in, uint16_t* qn,
-                              uint16_t* kn, uint16_t* qp, uint16_t* kp, uint16_t* vp, uint16_t* op, uint16_t* out,
+                              const int32_t* sample_idx, int n, const uint8_t* head_kind_in, uint16_t* kn,
+                              uint16_t* qp, uint16_t* kp, uint16_t* vp, uint16_t* op, uint16_t* out,
                               uint8_t* head_kind_out, float* mse_out, int32_t* row_ptr, int32_t* col, uint8_t* full,
                               int64_t capacity, void* workspace, size_t workspace_bytes, void* stream) {
   svg_status st;
   if (!head_kind_out) return SVG_ERR_INVALID_ARG;
-  if ((st = svg_qknorm_rope_layout(s, p, SVG_NORM_ROPE, q, k, nullptr, gamma_q, gamma_k, rope_table, nullptr, qn, kn,
-                                   nullptr, stream)) != SVG_OK)
+  // 1. QK-Norm + RoPE of K (profiling reads every normalised key)
+  if ((st = svg_qknorm_rope_layout(s, p, SVG_NORM_ROPE, nullptr, k, nullptr, nullptr, gamma_k, rope_table, nullptr,
+                                   nullptr, kn, nullptr, stream)) != SVG_OK)
     return st;
+  // 2. profiling; the sampled Q rows are normalised inside the kernel, with the same routine
   const uint8_t* kinds = head_kind_in;
   if (!kinds) {
-    if ((st = svg_profile_heads(s, p, qn, kn, v, sample_idx, n, workspace, workspace_bytes, mse_out, head_kind_out,
-                                stream)) != SVG_OK)
+    if ((st = svg_profile_heads_raw_q(s, p, q, gamma_q, rope_table, kn, v, sample_idx, n, workspace, workspace_bytes,
+                                      mse_out, head_kind_out, stream)) != SVG_OK)
       return st;
     kinds = head_kind_out;
   }
+  // 3. block index
   if ((st = svg_build_block_index(s, p, kinds, row_ptr, col, full, capacity, stream)) != SVG_OK) return st;
-  if ((st = svg_qknorm_rope_layout(s, p, SVG_LAYOUT, qn, kn, v, nullptr, nullptr, nullptr, kinds, qp, kp, vp,
-                                   stream)) != SVG_OK)
+  // 4. one pass: QK-Norm + RoPE of Q, and all three tensors into the heads' layouts
+  if ((st = svg_qknorm_rope_layout(s, p, SVG_NORM_ROPE | SVG_LAYOUT, q, kn, v, gamma_q, nullptr, rope_table, kinds,
+                                   qp, kp, vp, stream)) != SVG_OK)
     return st;
-  if (!op)   // attention writes the model-order output directly (inverse layout in its epilogue)
+  // 5. attention, with the inverse layout in its epilogue unless the head-layout output is wanted
+  if (!op)
     return svg_block_sparse_attn_model_order(s, p, qp, kp, vp, kinds, row_ptr, col, full, out, nullptr, stream);
   if ((st = svg_block_sparse_attn(s, p, qp, kp, vp, kinds, row_ptr, col, full, op, nullptr, stream)) != SVG_OK)
     return st;

@@ -341,3 +341,42 @@ def test_layer_schedule_dense_then_profiled_then_reused():
         ref = oracle.attention_rows(sh, pr, kinds, qn, kn, inp["v"], rows)
         assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, f"step {t}")
     assert np.array_equal(layer.kinds.cpu().numpy(), kinds_ref)
+
+
+# ------------------------------------------- five-pass step building blocks
+
+@pytest.mark.parametrize("key", ["cfg0", "ragged128", "smallS", "oddsplit", "cfg2"])
+def test_selective_norm_passes_match_the_two_stage_path(key):
+    """K alone, and {raw Q normalised + K, V moved} in one pass, give the same
+    bits as normalising both and then moving all three."""
+    wl, inp, _, _ = case(key)
+    pb = pb_of(wl)
+    table = torch.from_numpy(svg.rope_table(pb)).cuda()
+    q, k, v = dev(inp["q"]), dev(inp["k"]), dev(inp["v"])
+    gq, gk = dev(inp["gamma_q"]), dev(inp["gamma_k"])
+    kd = dev(mixed_kinds(wl.H))
+    qn, kn = svg.qknorm_rope(pb, q, k, gq, gk, table)
+    ref = svg.layout(pb, qn, kn, v, kd)
+    _, kn_only, _ = svg.qknorm_rope_layout(pb, None, k, None, None, gk, table, None, 1)
+    fused = svg.qknorm_rope_layout(pb, q, kn_only, v, gq, None, table, kd, 3)
+    svg.sync_status()
+    assert torch.equal(kn_only.view(torch.int16), kn.view(torch.int16))
+    for a, b in zip(fused, ref):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.parametrize("key", ["cfg0", "ragged128", "smallS128", "oddsplit", "cfg2"])
+def test_profile_raw_q_equals_profile_on_normalised_q(key):
+    """The sampled rows normalised inside the profiling kernel are the rows the
+    norm pass writes, so kinds and MSEs agree bit for bit."""
+    wl, inp, _, _ = case(key)
+    pb = pb_of(wl)
+    table = torch.from_numpy(svg.rope_table(pb)).cuda()
+    q, k, v = dev(inp["q"]), dev(inp["k"]), dev(inp["v"])
+    gq, gk, si = dev(inp["gamma_q"]), dev(inp["gamma_k"]), dev(inp["sample_idx"])
+    qn, kn = svg.qknorm_rope(pb, q, k, gq, gk, table)
+    kinds_a, mse_a = svg.profile_heads(pb, qn, kn, v, si)
+    kinds_b, mse_b = svg.profile_heads_raw_q(pb, q, gq, table, kn, v, si)
+    svg.sync_status()
+    assert torch.equal(kinds_a, kinds_b)
+    assert torch.equal(mse_a.view(torch.int32), mse_b.view(torch.int32))
