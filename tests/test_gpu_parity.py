@@ -55,9 +55,11 @@ CASES = {
     "wide": W.small_workload(d=64, H=2, F=5, Hs=6, Ws=7, T=9, w=4, r=41, n_samples=8),
     # RoPE sections not multiples of 8 wide: a lane's 4 pairs straddle two sections
     "oddsplit": W.small_workload(d=64, H=2, F=4, Hs=5, Ws=6, T=3, w=1, r=4, n_samples=8, rope_split=(18, 22, 24)),
+    # two batch entries: every per-head index runs over b*H + h
+    "batch2": W.small_workload(B=2, d=128, H=2, F=3, Hs=4, Ws=6, T=5, w=1, r=3, n_samples=8, bq=128),
 }
 FULL_ROW_CASES = ("cfg0", "ragged128", "tiny64", "smallS", "smallS128", "smallS_T0", "oneframe", "wide",
-                  "oddsplit")
+                  "oddsplit", "batch2")
 
 
 def pb_of(wl):
@@ -78,7 +80,7 @@ def rows_for(key, wl):
 
 # ------------------------------------------------------------ QK-Norm + RoPE
 
-@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "ragged128", "tiny64", "oneframe", "oddsplit"])
+@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "ragged128", "tiny64", "oneframe", "oddsplit", "batch2"])
 def test_qknorm_rope_within_one_ulp(key):
     wl, inp, qn_ref, kn_ref = case(key)
     pb = pb_of(wl)
@@ -106,12 +108,12 @@ def test_qknorm_rope_cfg3_sampled_rows():
 
 # ------------------------------------------------------------------ layout
 
-@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "ragged128", "tiny64", "smallS", "oneframe"])
+@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "ragged128", "tiny64", "smallS", "oneframe", "batch2"])
 def test_layout_and_inverse_bit_exact(key):
     wl, inp, _, _ = case(key)
     pb = pb_of(wl)
     sh = oracle.shape_of(wl)
-    kinds = mixed_kinds(wl.H)
+    kinds = mixed_kinds(wl.B * wl.H)
     q, k, v = dev(inp["q"]), dev(inp["k"]), dev(inp["v"])
     qp, kp, vp = svg.layout(pb, q, k, v, dev(kinds))
     back = svg.inverse_layout(pb, dev(kinds), qp)
@@ -128,7 +130,7 @@ def test_fused_norm_rope_layout(key):
     """flags = NORM_ROPE | LAYOUT equals the two separate passes bit for bit."""
     wl, inp, _, _ = case(key)
     pb = pb_of(wl)
-    kinds = dev(mixed_kinds(wl.H))
+    kinds = dev(mixed_kinds(wl.B * wl.H))
     args = (dev(inp["q"]), dev(inp["k"]))
     g = (dev(inp["gamma_q"]), dev(inp["gamma_k"]), dev(svg.rope_table(pb)))
     qn, kn = svg.qknorm_rope(pb, *args, *g)
@@ -149,12 +151,13 @@ def csr_host(row_ptr, col, full):
 
 @pytest.mark.parametrize("key,kinds_mode", [("cfg0", "mixed"), ("cfg1", "mixed"), ("cfg2", "mixed"),
                                             ("ragged128", "mixed"), ("tiny64", "mixed"), ("smallS", "mixed"),
-                                            ("oneframe", "mixed"), ("wide", "mixed"), ("cfg3", "planted")])
+                                            ("oneframe", "mixed"), ("wide", "mixed"), ("batch2", "mixed"),
+                                            ("cfg3", "planted")])
 def test_block_index_bit_exact(key, kinds_mode):
     wl = CASES[key]
     pb = pb_of(wl)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
-    kinds = mixed_kinds(wl.H) if kinds_mode == "mixed" else \
+    kinds = mixed_kinds(wl.B * wl.H) if kinds_mode == "mixed" else \
         np.array([W.SPATIAL if c == "S" else W.TEMPORAL for c in wl.planted], np.uint8)
     rp, col, full = csr_host(*svg.build_block_index(pb, dev(kinds)))
     svg.sync_status()
@@ -183,7 +186,8 @@ def test_block_index_capacity_overflow_is_reported():
 
 # --------------------------------------------------------------- profiling
 
-@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "smallS", "smallS128", "smallS_T0", "ragged128", "cfg3"])
+@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "smallS", "smallS128", "smallS_T0", "ragged128", "batch2",
+                                 "cfg3"])
 def test_profile_choices_bit_exact(key):
     wl, inp, qn, kn = case(key)
     pb = pb_of(wl)
@@ -234,13 +238,13 @@ def run_sparse(wl, qn, kn, v, kinds, want_lse=False, model_order=False):
 
 
 @pytest.mark.parametrize("key", ["cfg0", "ragged128", "tiny64", "smallS", "smallS128", "smallS_T0", "oneframe", "wide",
-                                 "cfg1", "cfg2"])
+                                 "batch2", "cfg1", "cfg2"])
 @pytest.mark.parametrize("kinds_mode", ["mixed", "spatial", "temporal"])
 def test_attention_parity(key, kinds_mode):
     wl, inp, qn, kn = case(key)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
-    kinds = {"mixed": mixed_kinds(wl.H), "spatial": np.zeros(wl.H, np.uint8),
-             "temporal": np.ones(wl.H, np.uint8)}[kinds_mode]
+    kinds = {"mixed": mixed_kinds(wl.B * wl.H), "spatial": np.zeros(wl.B * wl.H, np.uint8),
+             "temporal": np.ones(wl.B * wl.H, np.uint8)}[kinds_mode]
     out, lse = run_sparse(wl, qn, kn, inp["v"], kinds, want_lse=True)
     rows = rows_for(key, wl)
     ref, ref_lse = oracle.attention_rows(sh, pr, kinds, qn, kn, inp["v"], rows, want_lse=True)
@@ -259,7 +263,7 @@ def test_attention_model_order_equals_inverse_layout_pass(key):
     the bits the separate pass produces, and the LSE at the same positions."""
     wl, inp, qn, kn = case(key)
     sh = oracle.shape_of(wl)
-    kinds = mixed_kinds(wl.H)
+    kinds = mixed_kinds(wl.B * wl.H)
     out_a, lse_a = run_sparse(wl, qn, kn, inp["v"], kinds, want_lse=True)
     out_b, lse_b = run_sparse(wl, qn, kn, inp["v"], kinds, want_lse=True, model_order=True)
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
@@ -292,8 +296,8 @@ def test_attention_cfg3_sampled_rows():
 
 # ---------------------------------------------------------------- full step
 
-@pytest.mark.parametrize("key,head_layout_out", [("cfg0", False), ("smallS", False), ("cfg1", False),
-                                                  ("cfg2", False), ("cfg0", True), ("cfg2", True)])
+@pytest.mark.parametrize("key,head_layout_out", [("cfg0", False), ("smallS", False), ("batch2", False),
+                                                  ("cfg1", False), ("cfg2", False), ("cfg0", True), ("cfg2", True)])
 def test_full_step_end_to_end(key, head_layout_out):
     wl, inp, qn, kn = case(key)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
@@ -337,7 +341,7 @@ def test_layer_schedule_dense_then_profiled_then_reused():
         out = layer(t, *args)
         svg.sync_status()
         assert layer.last_mode == modes[t]
-        kinds = np.full(wl.H, W.DENSE, np.uint8) if t == 0 else kinds_ref
+        kinds = np.full(wl.B * wl.H, W.DENSE, np.uint8) if t == 0 else kinds_ref
         ref = oracle.attention_rows(sh, pr, kinds, qn, kn, inp["v"], rows)
         assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, f"step {t}")
     assert np.array_equal(layer.kinds.cpu().numpy(), kinds_ref)
@@ -354,7 +358,7 @@ def test_selective_norm_passes_match_the_two_stage_path(key):
     table = torch.from_numpy(svg.rope_table(pb)).cuda()
     q, k, v = dev(inp["q"]), dev(inp["k"]), dev(inp["v"])
     gq, gk = dev(inp["gamma_q"]), dev(inp["gamma_k"])
-    kd = dev(mixed_kinds(wl.H))
+    kd = dev(mixed_kinds(wl.B * wl.H))
     qn, kn = svg.qknorm_rope(pb, q, k, gq, gk, table)
     ref = svg.layout(pb, qn, kn, v, kd)
     _, kn_only, _ = svg.qknorm_rope_layout(pb, None, k, None, None, gk, table, None, 1)
