@@ -254,7 +254,7 @@ def run_gpu(args, rank, world, local_rank):
     # ---- end to end through the public host-buffer API (copies inside the timed region)
     out_h = torch.empty(q_h.shape, dtype=torch.bfloat16, pin_memory=True)
     for _ in range(2):
-        svg.sparse_attention(pb, q_h, k_h, v_h, gq_h, gk_h, si_h, buf, out_h)
+        svg.sparse_attention(pb, q_h, k_h, v_h, gq_h, gk_h, si_h, out_host=out_h)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -262,7 +262,7 @@ def run_gpu(args, rank, world, local_rank):
     e2e_steps = max(1, min(args.steps, 5))
     e0.record(stream)
     for _ in range(e2e_steps):
-        svg.sparse_attention(pb, q_h, k_h, v_h, gq_h, gk_h, si_h, buf, out_h)
+        svg.sparse_attention(pb, q_h, k_h, v_h, gq_h, gk_h, si_h, out_host=out_h)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps

@@ -9,7 +9,7 @@ from .api import (DENSE, SPATIAL, TEMPORAL, Problem, StepBuffers, attention_step
                   block_index_capacity, block_sparse_attn, build_block_index, inverse_layout, layout,
                   profile_heads, profile_heads_noalloc, profile_heads_raw_q, profile_workspace_size, qknorm_rope, qknorm_rope_layout, rope_table,
                   sample_queries, sparse_attention, sync_status)
-from .api import STEP_DENSE, STEP_PROFILE, STEP_REUSE, SparseAttentionLayer, step_policy  # noqa: F401
+from .api import STEP_DENSE, STEP_PROFILE, STEP_REUSE, HostPipeline, SparseAttentionLayer, step_policy  # noqa: F401
 
 __all__ = [
     "SVGError", "lib", "Problem", "StepBuffers", "SPATIAL", "TEMPORAL", "DENSE",
@@ -17,5 +17,5 @@ __all__ = [
     "build_block_index",
     "block_sparse_attn", "inverse_layout", "attention_step", "sparse_attention",
     "sample_queries", "rope_table", "block_index_capacity", "profile_workspace_size", "sync_status",
-    "STEP_DENSE", "STEP_PROFILE", "STEP_REUSE", "step_policy", "SparseAttentionLayer",
+    "STEP_DENSE", "STEP_PROFILE", "STEP_REUSE", "step_policy", "SparseAttentionLayer", "HostPipeline",
 ]

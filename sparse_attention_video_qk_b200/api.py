@@ -7,7 +7,7 @@ sm_100a kernels.  PyTorch provides device memory and streams.
 from __future__ import annotations
 
 import ctypes
-from dataclasses import dataclass
+from dataclasses import dataclass, replace
 
 import numpy as np
 import torch
@@ -282,26 +282,93 @@ def attention_step(pb: Problem, q, k, v, gamma_q, gamma_k, sample_idx, buffers: 
     return b.out
 
 
-def sparse_attention(pb: Problem, q_host, k_host, v_host, gamma_q, gamma_k, sample_idx, buffers: StepBuffers = None,
-                     out_host=None, device="cuda", stream=None):
-    """End-to-end call on host tensors: copies Q/K/V (bf16 [B,H,L,d], pinned for
-    asynchronous copies), gamma and the sample in, runs the step, copies O back
-    into `out_host` (allocated pinned if None).  Returns out_host."""
-    if buffers is None:
-        buffers = StepBuffers(pb, int(sample_idx.numel()), device)
-    s = stream if stream is not None else torch.cuda.current_stream()
-    with torch.cuda.stream(s):
-        q = q_host.to(device, non_blocking=True)
-        k = k_host.to(device, non_blocking=True)
-        v = v_host.to(device, non_blocking=True)
-        gq = gamma_q.to(device, non_blocking=True)
-        gk = gamma_k.to(device, non_blocking=True)
-        si = sample_idx.to(device, non_blocking=True)
-        o = attention_step(pb, q, k, v, gq, gk, si, buffers, stream=s)
+class HostPipeline:
+    """The step on host tensors with the host<->device copies overlapped with
+    the computation.  The B*H heads are split into `chunks` groups: group i+1
+    is copied in (one stream) while group i runs the five passes (a second
+    stream), and each group's output is copied out (a third stream) while the
+    next group runs.  Every stage is per head (profiling scores each head on
+    the shared sample), so the output equals the one-shot step bit for bit.
+    Device inputs and the output are full-size; the step's intermediates are
+    per group and reused."""
+
+    def __init__(self, pb: Problem, n_samples: int, chunks: int = 8, device="cuda"):
+        bh = pb.B * pb.H
+        chunks = max(1, min(int(chunks), bh))
+        base, extra = divmod(bh, chunks)
+        self.bounds = []
+        h = 0
+        for i in range(chunks):
+            n = base + (1 if i < extra else 0)
+            self.bounds.append((h, h + n))
+            h += n
+        self.pb, self.bh, self.n = pb, bh, n_samples
+        self.probs = {n: replace(pb, B=1, H=n) for n in {h1 - h0 for h0, h1 in self.bounds}}
+        self.bufs = {n: StepBuffers(p, n_samples, device) for n, p in self.probs.items()}
+        shp = (bh, pb.L, pb.d)
+        self.q, self.k, self.v, self.out = (torch.empty(shp, dtype=torch.bfloat16, device=device) for _ in range(4))
+        self.gq = torch.empty(pb.d, dtype=torch.float32, device=device)
+        self.gk = torch.empty(pb.d, dtype=torch.float32, device=device)
+        self.si = torch.empty(n_samples, dtype=torch.int32, device=device)
+        self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(device=device) for _ in range(3))
+
+    def __call__(self, q_host, k_host, v_host, gamma_q, gamma_k, sample_idx, out_host=None):
+        pb, bh = self.pb, self.bh
         if out_host is None:
-            out_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        out_host.copy_(o, non_blocking=True)
-    return out_host
+            out_host = torch.empty(q_host.shape, dtype=torch.bfloat16, pin_memory=True)
+        flat = lambda t: t.reshape(bh, pb.L, pb.d)
+        qh, kh, vh, oh = flat(q_host), flat(k_host), flat(v_host), flat(out_host)
+        caller = torch.cuda.current_stream()
+        # inputs are overwritten only after the previous call's passes are done
+        self.s_in.wait_stream(caller)
+        self.s_in.wait_stream(self.s_comp)
+        ev_in = []
+        with torch.cuda.stream(self.s_in):
+            self.gq.copy_(gamma_q, non_blocking=True)
+            self.gk.copy_(gamma_k, non_blocking=True)
+            self.si.copy_(sample_idx, non_blocking=True)
+            for h0, h1 in self.bounds:
+                self.q[h0:h1].copy_(qh[h0:h1], non_blocking=True)
+                self.k[h0:h1].copy_(kh[h0:h1], non_blocking=True)
+                self.v[h0:h1].copy_(vh[h0:h1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(self.s_in)
+                ev_in.append(ev)
+        # the output rows of a group are read back only after its passes
+        self.s_out.wait_stream(caller)
+        for (h0, h1), ev in zip(self.bounds, ev_in):
+            n = h1 - h0
+            b = self.bufs[n]
+            self.s_comp.wait_event(ev)
+            b.out = self.out[h0:h1]
+            attention_step(self.probs[n], self.q[h0:h1], self.k[h0:h1], self.v[h0:h1], self.gq, self.gk, self.si,
+                           b, stream=self.s_comp)
+            done = torch.cuda.Event()
+            done.record(self.s_comp)
+            self.s_out.wait_event(done)
+            with torch.cuda.stream(self.s_out):
+                oh[h0:h1].copy_(self.out[h0:h1], non_blocking=True)
+        caller.wait_stream(self.s_out)
+        return out_host
+
+
+_PIPELINES = {}
+
+
+def sparse_attention(pb: Problem, q_host, k_host, v_host, gamma_q, gamma_k, sample_idx, out_host=None,
+                     device="cuda", chunks: int = 8, pipeline: HostPipeline = None):
+    """End-to-end call on host tensors: Q/K/V (bf16 [B,H,L,d], pinned so the
+    copies are asynchronous), gamma and the sample go in, O comes back in
+    `out_host` (allocated pinned if None).  The copies overlap the passes
+    through a HostPipeline of `chunks` head groups (created once per shape and
+    cached, or passed in).  Work is ordered after the current stream, and the
+    current stream waits for the last copy.  Returns out_host."""
+    if pipeline is None:
+        key = (pb, int(sample_idx.numel()), int(chunks), str(device))
+        pipeline = _PIPELINES.get(key)
+        if pipeline is None:
+            pipeline = _PIPELINES[key] = HostPipeline(pb, int(sample_idx.numel()), chunks, device)
+    return pipeline(q_host, k_host, v_host, gamma_q, gamma_k, sample_idx, out_host)
 
 
 # ------------------------------------------------------ denoising schedule --
