@@ -110,42 +110,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x on the FMA pipe for a pair (x <= 8): x = n + f with n = round(x) and
-// f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients
-// minimise the maximum relative error on that interval (Remez exchange, see
-// gen_exp2_poly.py; max relative error 7.5e-5, far below bf16's 2^-8); 2^n
-// is added to the exponent field.  The rounding uses the 1.5 * 2^23 shift:
-// the integer n lands in the low mantissa bits of t, and (bits(t) << 23) is
-// n << 23.  x is clamped at -125 so the result stays a normal float
-// (2^-125 ~ 2.4e-38 stands in for 0 on masked keys).
-#ifndef SVG_POLY_EVERY
-#define SVG_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = SVG_POLY_EVERY;   // every kPolyEvery-th pair uses the polynomial (0: never)
-constexpr int kPolyStride = kPolyEvery > 0 ? kPolyEvery : 1;
-
-__device__ __forceinline__ void poly_exp2x2(float x0, float x1, float& p0, float& p1) {
-  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
-  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
-  constexpr float c2 = 0.2426111251115799f, c3 = 0.0551716685295105f;
-  x0 = fmaxf(x0, -125.0f);
-  x1 = fmaxf(x1, -125.0f);
-  const uint64_t x = f32x2(x0, x1);
-  const uint64_t t = fadd2(x, f32x2(kShift, kShift));
-  uint64_t n;
-  asm("sub.f32x2 %0, %1, %2;" : "=l"(n) : "l"(t), "l"(f32x2(kShift, kShift)));
-  uint64_t f;
-  asm("sub.f32x2 %0, %1, %2;" : "=l"(f) : "l"(x), "l"(n));
-  uint64_t q = ffma2(f32x2(c3, c3), f, f32x2(c2, c2));
-  q = ffma2(q, f, f32x2(c1, c1));
-  q = ffma2(q, f, f32x2(c0, c0));
-  float q0, q1, t0, t1;
-  unpack2(q, q0, q1);
-  unpack2(t, t0, t1);
-  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
-}
-
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
@@ -412,23 +376,14 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       const float msub = (m_use == -INFINITY) ? 0.f : m_use;
       const uint64_t nmsub2 = f32x2(-msub, -msub);
       // P = 2^(S*scale*log2e - m): the argument as packed fp32 pairs, 2^x on the
-      // MUFU unit except for every kPolyEvery-th pair (FMA-pipe polynomial);
-      // row sum over 8 independent packed chains
+      // MUFU unit; row sum over 8 independent packed chains
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < 64; c++) {
         const uint64_t xa = ffma2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2x2, nmsub2);
         float x0, x1;
         unpack2(xa, x0, x1);
-        float p0, p1;
-        bool use_poly = false;
-        if constexpr (kPolyEvery > 0) use_poly = (c % kPolyStride) == kPolyStride - 1;
-        if (use_poly) {
-          poly_exp2x2(x0, x1, p0, p1);
-        } else {
-          p0 = fast_exp2(x0);
-          p1 = fast_exp2(x1);
-        }
+        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
         acc[c & 3] = fadd2(acc[c & 3], f32x2(p0, p1));
         sr[c] = pack_bf16x2(p0, p1);
       }
