@@ -287,6 +287,13 @@ size_t svg_profile_workspace_size(const svg_shape* shape, int n);
  * synchronisation itself failed). */
 svg_status svg_sync_status(void* stream);
 
+/* Failure-path self-test (not on the pages): launches one warp that waits on a
+ * barrier nothing completes.  The wait gives up after its limit (about a
+ * second), records SVG_ERR_TIMEOUT in the error word and returns, exactly as a
+ * stalled pipeline in any kernel of this library would; the context stays
+ * usable.  svg_sync_status(stream) then reports SVG_ERR_TIMEOUT and clears it. */
+svg_status svg_selftest_wait_timeout(void* stream);
+
 const char* svg_status_string(svg_status status);
 const char* svg_version(void);
 

@@ -217,6 +217,21 @@ svg_status launch_profile(const svg_shape* s, const svg_params* p, const uint16_
   return launch_status();
 }
 
+// Self-test of the bounded wait: one warp waits on an mbarrier that nothing
+// completes.  After the wait limit (about a second) mbar_wait records
+// kErrTimeout in the error word and returns false; the kernel then returns.
+__global__ void selftest_wait_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&bar), 1);
+    abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(smem_addr(&bar), 0, &abort_flag);
+}
+
 }  // namespace
 
 // ===================================================================== ABI
@@ -329,6 +344,11 @@ size_t svg_profile_workspace_size(const svg_shape* s, int n) {
   if (check_shape(s) != SVG_OK || n <= 0) return 0;
   const int BH = s->B * s->H;
   return prof_workspace_bytes(BH, s->L, s->d, prof_chunks(BH, s->L));
+}
+
+svg_status svg_selftest_wait_timeout(void* stream) {
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return launch_status();
 }
 
 svg_status svg_sync_status(void* stream) {
