@@ -36,10 +36,11 @@ constexpr int kProfKeys = 128;     // keys per tile
 // (stored field-major per chunk: [chunk][field][lane]).
 __host__ __device__ constexpr int prof_rec_floats(int D) { return 3 + 2 * D; }
 
-// Key chunks per head: about 2 waves of 148 SMs, at least two tiles each.
+// Key chunks per head: as many as fit in 2 full waves of 148 SMs (one CTA per
+// SM), so no partial third wave, and at least two tiles each.
 __host__ __device__ inline int prof_chunks(int BH, int L) {
   const int ntiles = (L + kProfKeys - 1) / kProfKeys;
-  int c = (2 * 148 + BH - 1) / BH;
+  int c = (2 * 148) / BH;
   const int cap = (ntiles + 1) / 2;
   if (c > cap) c = cap;
   if (c < 1) c = 1;
