@@ -292,14 +292,18 @@ class HostPipeline:
     Device inputs and the output are full-size; the step's intermediates are
     per group and reused."""
 
-    def __init__(self, pb: Problem, n_samples: int, chunks: int = 8, device="cuda"):
+    def __init__(self, pb: Problem, n_samples: int, chunks: int = 8, device="cuda", sizes=None):
         bh = pb.B * pb.H
-        chunks = max(1, min(int(chunks), bh))
-        base, extra = divmod(bh, chunks)
+        if sizes is None:
+            chunks = max(1, min(int(chunks), bh))
+            base, extra = divmod(bh, chunks)
+            sizes = [base + (1 if i < extra else 0) for i in range(chunks)]
+        sizes = [int(n) for n in sizes]
+        if sum(sizes) != bh or min(sizes) < 1:
+            raise ValueError(f"group sizes {sizes} must be positive and sum to B*H = {bh}")
         self.bounds = []
         h = 0
-        for i in range(chunks):
-            n = base + (1 if i < extra else 0)
+        for n in sizes:
             self.bounds.append((h, h + n))
             h += n
         self.pb, self.bh, self.n = pb, bh, n_samples

@@ -313,14 +313,15 @@ def test_full_step_end_to_end(key, head_layout_out):
     assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, key)
 
 
-@pytest.mark.parametrize("key,chunks", [("cfg2", 4), ("cfg2", 5), ("batch2", 3), ("cfg0", 1)])
+@pytest.mark.parametrize("key,chunks", [("cfg2", 4), ("cfg2", 5), ("batch2", 3), ("cfg0", 1), ("batch2", [1, 2, 1])])
 def test_host_pipeline_chunks_match_one_shot_step(key, chunks):
     """Head groups copied in, computed and copied out on three streams give
     the one-shot device step's bits, for even and uneven groups and B > 1."""
     wl, inp, _, _ = case(key)
     pb = pb_of(wl)
     pin = lambda a: torch.from_numpy(a).view(torch.bfloat16).pin_memory()
-    pipe = svg.HostPipeline(pb, wl.n_samples, chunks=chunks)
+    pipe = (svg.HostPipeline(pb, wl.n_samples, sizes=chunks) if isinstance(chunks, list)
+            else svg.HostPipeline(pb, wl.n_samples, chunks=chunks))
     args = (pin(inp["q"]), pin(inp["k"]), pin(inp["v"]), torch.from_numpy(inp["gamma_q"]).pin_memory(),
             torch.from_numpy(inp["gamma_k"]).pin_memory(), torch.from_numpy(inp["sample_idx"]).pin_memory())
     out_h = pipe(*args)
