@@ -3,6 +3,22 @@
 The library ``libsvg_b200.so`` (C ABI: include/svg.h) holds every kernel;
 this package is its Python binding.  Build the library with
 ``python -m sparse_attention_video_qk_b200.build``.
+
+Typical use, one layer of a video DiT (tensors bf16 [B, H, L, d] on the GPU,
+video tokens frame-major and text tokens after them)::
+
+    import sparse_attention_video_qk_b200 as svg
+    pb = svg.Problem(B=1, H=24, d=128, F=33, Hs=45, Ws=80, text_len=256,
+                     spatial_frames=1, temporal_radius=256)
+    buf = svg.StepBuffers(pb, n_samples=64)                 # allocated once, reused
+    sample = torch.from_numpy(svg.sample_queries(seed, pb.Lv, 64)).cuda()
+    out = svg.attention_step(pb, q, k, v, gamma_q, gamma_k, sample, buf)
+
+``SparseAttentionLayer`` adds the denoising schedule (dense for the first
+quarter of the steps, then profiled), and ``sparse_attention`` /
+``HostPipeline`` take pinned host tensors and overlap the copies with the
+computation.  Each stage is also callable on its own (``qknorm_rope_layout``,
+``profile_heads``, ``build_block_index``, ``block_sparse_attn``, ...).
 """
 from ._lib import SVGError, lib  # noqa: F401
 from .api import (DENSE, SPATIAL, TEMPORAL, Problem, StepBuffers, attention_step,  # noqa: F401
