@@ -35,6 +35,14 @@ def case(key):
     return wl, inp, qn, kn
 
 
+@functools.lru_cache(maxsize=None)
+def profile_ref(key):
+    """Oracle profiling of a named case: (mse [BH, 2], kinds [BH]) (cached)."""
+    wl, inp, qn, kn = case(key)
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    return oracle.profile(sh, pr, qn, kn, inp["v"], inp["sample_idx"])
+
+
 CASES = {
     "cfg0": W.CONFIGS[0],
     "cfg1": W.CONFIGS[1],
@@ -192,7 +200,7 @@ def test_profile_choices_bit_exact(key):
     wl, inp, qn, kn = case(key)
     pb = pb_of(wl)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
-    mse_ref, kinds_ref = oracle.profile(sh, pr, qn, kn, inp["v"], inp["sample_idx"])
+    mse_ref, kinds_ref = profile_ref(key)
     kinds, mse = svg.profile_heads(pb, dev(qn), dev(kn), dev(inp["v"]), dev(inp["sample_idx"]))
     svg.sync_status()
     kinds = kinds.cpu().numpy()
@@ -297,8 +305,11 @@ def test_attention_cfg3_sampled_rows():
 # ---------------------------------------------------------------- full step
 
 @pytest.mark.parametrize("key,head_layout_out", [("cfg0", False), ("smallS", False), ("batch2", False),
-                                                  ("cfg1", False), ("cfg2", False), ("cfg0", True), ("cfg2", True)])
+                                                  ("cfg1", False), ("cfg2", False), ("cfg0", True), ("cfg2", True),
+                                                  ("cfg3", False)])
 def test_full_step_end_to_end(key, head_layout_out):
+    """The whole five-pass step (config 3: the workload and launches bench.py
+    times) against the oracle: head kinds bit-exact, sampled output rows."""
     wl, inp, qn, kn = case(key)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
     pb = pb_of(wl)
@@ -306,7 +317,7 @@ def test_full_step_end_to_end(key, head_layout_out):
     out = svg.attention_step(pb, dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["gamma_q"]),
                              dev(inp["gamma_k"]), dev(inp["sample_idx"]), buf)
     svg.sync_status()
-    _, kinds_ref = oracle.profile(sh, pr, qn, kn, inp["v"], inp["sample_idx"])
+    _, kinds_ref = profile_ref(key)
     assert np.array_equal(buf.kinds.cpu().numpy(), kinds_ref)
     rows = rows_for(key, wl)
     ref = oracle.attention_rows(sh, pr, kinds_ref, qn, kn, inp["v"], rows)
