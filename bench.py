@@ -34,6 +34,9 @@ sys.path.insert(0, ROOT)
 import svg_workloads as W  # noqa: E402
 
 METRIC = "sparse-attn layer ms and effective TFLOP/s (% bf16 peak) at 118,800 tokens"
+SHAPE_LABEL = {W.TINY.name: "tiny test shape", W.COGVIDEOX.name: "CogVideoX shape",
+               W.WAN.name: "Wan 2.1-1.3B shape", W.HUNYUAN.name: "HunyuanVideo 720p 5 s shape",
+               W.HUNYUAN_SWEEP.name: "HunyuanVideo 720p 5 s shape, sweep seed"}
 NOMINAL_BF16_TFLOPS = 2250.0
 NOMINAL_HBM_GBS = 7700.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -170,7 +173,7 @@ def run_gpu(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
-    wl = W.CONFIGS[args.config]
+    wl = W.WORKLOADS[args.workload]
     pb = svg.Problem.from_workload(wl)
     inp = W.make_inputs(wl, seed=wl.seed + rank)          # each rank: its own layer
     pin = lambda a, bf=True: (torch.from_numpy(a).view(torch.bfloat16) if bf else torch.from_numpy(a)).pin_memory()
@@ -301,7 +304,7 @@ def run_gpu(args, rank, world, local_rank):
     # svg_block_sparse_attn runs the two-query-tile kernel for 128-row tiles
     attn_src, attn_name = (("attention2.cuh", f"attn2_kernel<{wl.d}>") if wl.bq == 128
                            else ("attention.cuh", f"attn_kernel<{wl.d}>"))
-    traffic = traffic_from_profile(attn_src, "attention_hunyuan_cfg3.md") if args.config == 3 else None
+    traffic = traffic_from_profile(attn_src, "attention_hunyuanvideo_720p.md") if wl == W.HUNYUAN else None
     d, L, BH = wl.d, wl.L, wl.B * wl.H
     stage_bytes = {"k_norm_rope": 4.0 * BH * L * d, "q_norm_rope_layout": 12.0 * BH * L * d,
                    "profile": 4.0 * BH * L * d}
@@ -319,7 +322,7 @@ def run_gpu(args, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) Q/K/V with planted spatial/temporal heads; no model weights)",
         "config": {
-            "workload": f"{wl.name} (HunyuanVideo 720p 5 s shape)",
+            "workload": f"{wl.name} ({SHAPE_LABEL[wl.name]})",
             "B": wl.B, "H": wl.H, "d": wl.d, "frames": wl.F, "grid": f"{wl.Hs}x{wl.Ws}", "text_tokens": wl.T,
             "video_tokens": wl.Lv, "seq_len": wl.L, "spatial_window": wl.w, "temporal_radius": wl.r,
             "tile": f"{wl.bq}x{wl.bk}", "profiled_rows": wl.n_samples,
@@ -378,7 +381,7 @@ def token_density(wl, kind):
 
 
 def run_sweep(args):
-    """Forced-kind sweep at the config-3 shape: every head spatial with
+    """Forced-kind sweep at the HunyuanVideo shape: every head spatial with
     w in {0,1,2,4,8}, then every head temporal (layout applied) with r in
     {32,...,1800}; attention time against dense on the same inputs."""
     import torch
@@ -387,7 +390,7 @@ def run_sweep(args):
 
     device = torch.device("cuda", 0)
     torch.cuda.set_device(0)
-    base = W.CONFIGS[4]
+    base = W.HUNYUAN_SWEEP
     pb0 = svg.Problem.from_workload(base)
     g = torch.Generator(device=device).manual_seed(base.seed)
     shp = (base.B, base.H, base.L, base.d)
@@ -457,7 +460,7 @@ def oracle_sample_rate(wl, inp, n_rows: int, seed: int = 0):
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
     kinds = np.array([0 if c == "S" else 1 for c in wl.planted], np.uint8)
     rng = np.random.Generator(np.random.PCG64(seed))
-    per_head = max(1, n_rows // (wl.B * wl.H))
+    per_head = max(1, min(wl.L, n_rows // (wl.B * wl.H)))
     rows = np.concatenate([bh * wl.L + rng.choice(wl.L, per_head, replace=False) for bh in range(wl.B * wl.H)])
     # the attention rows need normalised Q rows and every normalised K row of their heads
     t0 = time.perf_counter()
@@ -515,7 +518,7 @@ def cpu_baseline(wl, inp, n_rows):
 def run_reference(args, rank):
     if rank != 0:
         return None
-    wl = W.CONFIGS[args.config]
+    wl = W.WORKLOADS[args.workload]
     inp = W.make_inputs(wl)
     rates, secs_all = [], []
     for s in range(args.warmup + args.steps):
@@ -529,7 +532,7 @@ def run_reference(args, rank):
         "metric": METRIC, "value": round(value, 8), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(1000 * statistics.mean(secs_all), 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": f"{wl.name} (HunyuanVideo 720p 5 s shape)", "B": wl.B, "H": wl.H, "d": wl.d,
+        "config": {"workload": f"{wl.name} ({SHAPE_LABEL[wl.name]})", "B": wl.B, "H": wl.H, "d": wl.d,
                    "seq_len": wl.L, "sampled_rows_per_step": args.ref_rows,
                    "kept_tile_gflop_per_step": round(flops_step / 1e9, 3)},
         "cpu_baseline": {"value": round(value, 8), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
@@ -546,7 +549,7 @@ def main():
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--config", type=int, default=3)
+    ap.add_argument("--workload", default=W.HUNYUAN.name, choices=sorted(W.WORKLOADS))
     ap.add_argument("--cpu-rows", type=int, default=14400)
     ap.add_argument("--ref-rows", type=int, default=960)
     ap.add_argument("--no-dense", action="store_true")

@@ -84,33 +84,34 @@ def _alt(H, pattern):
     return tuple(pattern[h % len(pattern)] for h in range(H))
 
 
-# The five configurations.  Block size is given only for configs 0 and 1; the
-# 128 x 64 tile of config 1 is used for the larger shapes as well.  The RoPE
-# split is given only for d = 64 (16:24:24); for d = 128 the same ratio
-# (32:48:48) is used.
-CONFIGS = {
-    0: Workload("tiny-f4-8x8", B=1, H=2, d=64, F=4, Hs=8, Ws=8, T=0, w=1, r=8, n_samples=16,
-                bq=64, bk=64, planted=("S", "T"), rope_split=(16, 24, 24), seed=1000),
-    1: Workload("cogvideox-f13-30x45", B=1, H=48, d=64, F=13, Hs=30, Ws=45, T=226, w=1, r=64,
-                n_samples=64, bq=128, bk=64, planted=_alt(48, "ST"), rope_split=(16, 24, 24),
-                seed=1001),
-    2: Workload("wan2.1-1.3b-f21-30x52", B=1, H=12, d=128, F=21, Hs=30, Ws=52, T=512, w=1, r=96,
-                n_samples=64, bq=128, bk=64, planted=_alt(12, "STU"), rope_split=(32, 48, 48),
-                seed=1002),
-    3: Workload("hunyuanvideo-720p-5s-f33-45x80", B=1, H=24, d=128, F=33, Hs=45, Ws=80, T=256,
-                w=1, r=256, n_samples=64, bq=128, bk=64, planted=_alt(24, "ST"),
-                rope_split=(32, 48, 48), seed=1003),
-}
-CONFIGS[4] = replace(CONFIGS[3], name="hunyuanvideo-sparsity-sweep", seed=1004)
+# The workloads.  Block size is given only for the tiny and CogVideoX shapes;
+# the 128 x 64 tile of the CogVideoX shape is used for the larger shapes as
+# well.  The RoPE split is given only for d = 64 (16:24:24); for d = 128 the
+# same ratio (32:48:48) is used.
+TINY = Workload("tiny-f4-8x8", B=1, H=2, d=64, F=4, Hs=8, Ws=8, T=0, w=1, r=8, n_samples=16,
+                bq=64, bk=64, planted=("S", "T"), rope_split=(16, 24, 24), seed=1000)
+COGVIDEOX = Workload("cogvideox-f13-30x45", B=1, H=48, d=64, F=13, Hs=30, Ws=45, T=226, w=1, r=64,
+                     n_samples=64, bq=128, bk=64, planted=_alt(48, "ST"), rope_split=(16, 24, 24),
+                     seed=1001)
+WAN = Workload("wan2.1-1.3b-f21-30x52", B=1, H=12, d=128, F=21, Hs=30, Ws=52, T=512, w=1, r=96,
+               n_samples=64, bq=128, bk=64, planted=_alt(12, "STU"), rope_split=(32, 48, 48),
+               seed=1002)
+HUNYUAN = Workload("hunyuanvideo-720p-5s-f33-45x80", B=1, H=24, d=128, F=33, Hs=45, Ws=80, T=256,
+                   w=1, r=256, n_samples=64, bq=128, bk=64, planted=_alt(24, "ST"),
+                   rope_split=(32, 48, 48), seed=1003)
+# the HunyuanVideo shape with the head kinds forced, one density per point
+HUNYUAN_SWEEP = replace(HUNYUAN, name="hunyuanvideo-sparsity-sweep", seed=1004)
 
-# Sweep points of config 4 (head kinds forced, so each point has one density).
+WORKLOADS = {w.name: w for w in (TINY, COGVIDEOX, WAN, HUNYUAN, HUNYUAN_SWEEP)}
+
+# Sweep points (head kinds forced, so each point has one density).
 SWEEP_SPATIAL_W = (0, 1, 2, 4, 8)
 SWEEP_TEMPORAL_R = (32, 64, 128, 256, 512, 900, 1800)
 
 
 def sweep_points():
-    """(label, workload) pairs of the config-4 sparsity sweep."""
-    base = CONFIGS[4]
+    """(label, workload) pairs of the sparsity sweep at the HunyuanVideo shape."""
+    base = HUNYUAN_SWEEP
     pts = []
     for w in SWEEP_SPATIAL_W:
         pts.append((f"spatial_w{w}", replace(base, w=w, forced_kinds=(SPATIAL,) * base.H)))

@@ -50,7 +50,7 @@ def test_sample_queries_matches_generator(L):
 
 
 def test_rope_table_values(L):
-    wl = W.CONFIGS[0]
+    wl = W.TINY
     pb = api.Problem.from_workload(wl)
     tab = api.rope_table(pb)
     n0, n1, n2 = wl.rope_split
@@ -66,7 +66,7 @@ def test_rope_table_values(L):
 
 
 def test_capacity_and_workspace(L):
-    wl = W.CONFIGS[3]
+    wl = W.HUNYUAN
     pb = api.Problem.from_workload(wl)
     assert api.block_index_capacity(pb) == wl.H * wl.nqb * wl.nkb
     ws = api.profile_workspace_size(pb, 64)
@@ -81,7 +81,7 @@ def _call_attn(L, sh, pr, ptr=16):
 
 def test_host_side_argument_errors(L):
     """Errors are returned before anything touches the GPU."""
-    pb = api.Problem.from_workload(W.CONFIGS[0])
+    pb = api.Problem.from_workload(W.TINY)
     sh, pr = pb.c_shape(), pb.c_params()
     bad = C.SvgShape(sh.B, sh.H, sh.L + 1, sh.d, sh.F, sh.Hs, sh.Ws, sh.text_len)
     assert _call_attn(L, bad, pr) == C.SVG_ERR_SHAPE
@@ -116,8 +116,8 @@ def test_noalloc_capacity_limit(L):
     """The no-alloc profiling entry rejects shapes whose one key chunk of
     partials does not fit its 16 MiB scratch, before any CUDA call."""
     p = ctypes.c_void_p(16)
-    for wl_idx, heads in ((2, 126), (1, 247)):          # d = 128: B*H > 125; d = 64: B*H > 246
-        pb = api.Problem.from_workload(W.CONFIGS[wl_idx])
+    for wl, heads in ((W.WAN, 126), (W.COGVIDEOX, 247)):   # d = 128: B*H > 125; d = 64: B*H > 246
+        pb = api.Problem.from_workload(wl)
         sh, pr = pb.c_shape(), pb.c_params()
         big = C.SvgShape(1, heads, sh.L, sh.d, sh.F, sh.Hs, sh.Ws, sh.text_len)
         per_chunk = heads * 128 * (3 + 2 * sh.d) * 4 + heads * 64 * 2 * 8

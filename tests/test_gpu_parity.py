@@ -44,10 +44,10 @@ def profile_ref(key):
 
 
 CASES = {
-    "cfg0": W.CONFIGS[0],
-    "cfg1": W.CONFIGS[1],
-    "cfg2": W.CONFIGS[2],
-    "cfg3": W.CONFIGS[3],
+    "tiny": W.TINY,
+    "cogvideox": W.COGVIDEOX,
+    "wan": W.WAN,
+    "hunyuan": W.HUNYUAN,
     # ragged: L = 116 is a multiple of neither tile size; text present; d = 128
     "ragged128": W.small_workload(d=128, H=3, F=3, Hs=5, Ws=7, T=11, w=1, r=6, n_samples=12, bq=128),
     # tiny: L = 11 < one tile
@@ -66,7 +66,7 @@ CASES = {
     # two batch entries: every per-head index runs over b*H + h
     "batch2": W.small_workload(B=2, d=128, H=2, F=3, Hs=4, Ws=6, T=5, w=1, r=3, n_samples=8, bq=128),
 }
-FULL_ROW_CASES = ("cfg0", "ragged128", "tiny64", "smallS", "smallS128", "smallS_T0", "oneframe", "wide",
+FULL_ROW_CASES = ("tiny", "ragged128", "tiny64", "smallS", "smallS128", "smallS_T0", "oneframe", "wide",
                   "oddsplit", "batch2")
 
 
@@ -81,14 +81,14 @@ def mixed_kinds(H):
 def rows_for(key, wl):
     if key in FULL_ROW_CASES:
         return np.arange(wl.B * wl.H * wl.L, dtype=np.int64)
-    if key == "cfg3":
+    if key == "hunyuan":
         return W.random_rows(wl, 48, seed=11, max_boundary_tiles=1)
     return W.random_rows(wl, 96, seed=11, max_boundary_tiles=3)
 
 
 # ------------------------------------------------------------ QK-Norm + RoPE
 
-@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "ragged128", "tiny64", "oneframe", "oddsplit", "batch2"])
+@pytest.mark.parametrize("key", ["tiny", "cogvideox", "wan", "ragged128", "tiny64", "oneframe", "oddsplit", "batch2"])
 def test_qknorm_rope_within_one_ulp(key):
     wl, inp, qn_ref, kn_ref = case(key)
     pb = pb_of(wl)
@@ -99,8 +99,8 @@ def test_qknorm_rope_within_one_ulp(key):
         assert_norm_rope_close(got, ref, f"{key}/{name}")
 
 
-def test_qknorm_rope_cfg3_sampled_rows():
-    wl = W.CONFIGS[3]
+def test_qknorm_rope_hunyuan_sampled_rows():
+    wl = W.HUNYUAN
     inp = W.make_inputs(wl)
     pb = pb_of(wl)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
@@ -116,7 +116,7 @@ def test_qknorm_rope_cfg3_sampled_rows():
 
 # ------------------------------------------------------------------ layout
 
-@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "ragged128", "tiny64", "smallS", "oneframe", "batch2"])
+@pytest.mark.parametrize("key", ["tiny", "cogvideox", "wan", "ragged128", "tiny64", "smallS", "oneframe", "batch2"])
 def test_layout_and_inverse_bit_exact(key):
     wl, inp, _, _ = case(key)
     pb = pb_of(wl)
@@ -133,7 +133,7 @@ def test_layout_and_inverse_bit_exact(key):
                           oracle.layout(sh, kinds, oracle.layout(sh, kinds, inp["v"]), inverse=True))
 
 
-@pytest.mark.parametrize("key", ["cfg0", "ragged128", "smallS"])
+@pytest.mark.parametrize("key", ["tiny", "ragged128", "smallS"])
 def test_fused_norm_rope_layout(key):
     """flags = NORM_ROPE | LAYOUT equals the two separate passes bit for bit."""
     wl, inp, _, _ = case(key)
@@ -157,10 +157,10 @@ def csr_host(row_ptr, col, full):
     return rp, col[:nnz].cpu().numpy(), full[:nnz].cpu().numpy()
 
 
-@pytest.mark.parametrize("key,kinds_mode", [("cfg0", "mixed"), ("cfg1", "mixed"), ("cfg2", "mixed"),
+@pytest.mark.parametrize("key,kinds_mode", [("tiny", "mixed"), ("cogvideox", "mixed"), ("wan", "mixed"),
                                             ("ragged128", "mixed"), ("tiny64", "mixed"), ("smallS", "mixed"),
                                             ("oneframe", "mixed"), ("wide", "mixed"), ("batch2", "mixed"),
-                                            ("cfg3", "planted")])
+                                            ("hunyuan", "planted")])
 def test_block_index_bit_exact(key, kinds_mode):
     wl = CASES[key]
     pb = pb_of(wl)
@@ -194,8 +194,8 @@ def test_block_index_capacity_overflow_is_reported():
 
 # --------------------------------------------------------------- profiling
 
-@pytest.mark.parametrize("key", ["cfg0", "cfg1", "cfg2", "smallS", "smallS128", "smallS_T0", "ragged128", "batch2",
-                                 "cfg3"])
+@pytest.mark.parametrize("key", ["tiny", "cogvideox", "wan", "smallS", "smallS128", "smallS_T0", "ragged128", "batch2",
+                                 "hunyuan"])
 def test_profile_choices_bit_exact(key):
     wl, inp, qn, kn = case(key)
     pb = pb_of(wl)
@@ -212,13 +212,13 @@ def test_profile_choices_bit_exact(key):
     rel = np.abs(mse - mse_ref) / mse_ref
     assert rel.max() < 2e-2, rel.max()
     planted = inp["planted"]
-    if key in ("cfg0", "cfg2", "cfg3"):
+    if key in ("tiny", "wan", "hunyuan"):
         sel = planted != 255
         assert np.array_equal(kinds[sel], planted[sel])
 
 
 def test_profile_bad_sample_index_reported():
-    wl, inp, qn, kn = case("cfg0")
+    wl, inp, qn, kn = case("tiny")
     pb = pb_of(wl)
     bad = inp["sample_idx"].copy()
     bad[3] = wl.L + 5
@@ -245,8 +245,8 @@ def run_sparse(wl, qn, kn, v, kinds, want_lse=False, model_order=False):
     return out, lse
 
 
-@pytest.mark.parametrize("key", ["cfg0", "ragged128", "tiny64", "smallS", "smallS128", "smallS_T0", "oneframe", "wide",
-                                 "batch2", "cfg1", "cfg2"])
+@pytest.mark.parametrize("key", ["tiny", "ragged128", "tiny64", "smallS", "smallS128", "smallS_T0", "oneframe", "wide",
+                                 "batch2", "cogvideox", "wan"])
 @pytest.mark.parametrize("kinds_mode", ["mixed", "spatial", "temporal"])
 def test_attention_parity(key, kinds_mode):
     wl, inp, qn, kn = case(key)
@@ -265,7 +265,7 @@ def test_attention_parity(key, kinds_mode):
     assert np.abs(lse_h[bh, pos] - ref_lse).max() < 5e-3
 
 
-@pytest.mark.parametrize("key", ["cfg0", "ragged128", "smallS128", "cfg2"])
+@pytest.mark.parametrize("key", ["tiny", "ragged128", "smallS128", "wan"])
 def test_attention_model_order_equals_inverse_layout_pass(key):
     """The inverse layout fused into the attention epilogue stores exactly
     the bits the separate pass produces, and the LSE at the same positions."""
@@ -292,23 +292,23 @@ def test_attention_dense_kinds_equal_dense_attention():
     assert_attention_close(host_bits(out).reshape(-1, wl.d), ref, MAX_ABS, MEAN_ABS, "dense")
 
 
-def test_attention_cfg3_sampled_rows():
-    wl, inp, qn, kn = case("cfg3")
+def test_attention_hunyuan_sampled_rows():
+    wl, inp, qn, kn = case("hunyuan")
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
     kinds = np.array([W.SPATIAL if c == "S" else W.TEMPORAL for c in wl.planted], np.uint8)
     out, _ = run_sparse(wl, qn, kn, inp["v"], kinds, model_order=True)     # the launch bench.py times
-    rows = rows_for("cfg3", wl)
+    rows = rows_for("hunyuan", wl)
     ref = oracle.attention_rows(sh, pr, kinds, qn, kn, inp["v"], rows)
-    assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, "cfg3")
+    assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, "hunyuan")
 
 
 # ---------------------------------------------------------------- full step
 
-@pytest.mark.parametrize("key,head_layout_out", [("cfg0", False), ("smallS", False), ("batch2", False),
-                                                  ("cfg1", False), ("cfg2", False), ("cfg0", True), ("cfg2", True),
-                                                  ("cfg3", False)])
+@pytest.mark.parametrize("key,head_layout_out", [("tiny", False), ("smallS", False), ("batch2", False),
+                                                  ("cogvideox", False), ("wan", False), ("tiny", True), ("wan", True),
+                                                  ("hunyuan", False)])
 def test_full_step_end_to_end(key, head_layout_out):
-    """The whole five-pass step (config 3: the workload and launches bench.py
+    """The whole five-pass step (the HunyuanVideo shape: the workload and launches bench.py
     times) against the oracle: head kinds bit-exact, sampled output rows."""
     wl, inp, qn, kn = case(key)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
@@ -324,7 +324,7 @@ def test_full_step_end_to_end(key, head_layout_out):
     assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, key)
 
 
-@pytest.mark.parametrize("key,chunks", [("cfg2", 4), ("cfg2", 5), ("batch2", 3), ("cfg0", 1), ("batch2", [1, 2, 1])])
+@pytest.mark.parametrize("key,chunks", [("wan", 4), ("wan", 5), ("batch2", 3), ("tiny", 1), ("batch2", [1, 2, 1])])
 def test_host_pipeline_chunks_match_one_shot_step(key, chunks):
     """Head groups copied in, computed and copied out on three streams give
     the one-shot device step's bits, for even and uneven groups and B > 1."""
@@ -347,7 +347,7 @@ def test_host_pipeline_chunks_match_one_shot_step(key, chunks):
 
 
 def test_host_buffer_api_matches_device_api():
-    wl, inp, _, _ = case("cfg0")
+    wl, inp, _, _ = case("tiny")
     pb = pb_of(wl)
     pin = lambda a: torch.from_numpy(a).view(torch.bfloat16).pin_memory()
     out_h = svg.sparse_attention(pb, pin(inp["q"]), pin(inp["k"]), pin(inp["v"]), torch.from_numpy(inp["gamma_q"]),
@@ -363,12 +363,12 @@ def test_host_buffer_api_matches_device_api():
 def test_layer_schedule_dense_then_profiled_then_reused():
     """SparseAttentionLayer over 4 denoising steps: step 0 dense, step 1
     profiled, step 2 reuses step 1's kinds, step 3 profiles again."""
-    wl, inp, qn, kn = case("cfg0")
+    wl, inp, qn, kn = case("tiny")
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
     layer = svg.SparseAttentionLayer(pb_of(wl), wl.n_samples, total_steps=4, dense_fraction=0.25, reprofile_every=2)
     args = tuple(dev(inp[k]) for k in ("q", "k", "v", "gamma_q", "gamma_k", "sample_idx"))
     _, kinds_ref = oracle.profile(sh, pr, qn, kn, inp["v"], inp["sample_idx"])
-    rows = rows_for("cfg0", wl)
+    rows = rows_for("tiny", wl)
     modes = [svg.STEP_DENSE, svg.STEP_PROFILE, svg.STEP_REUSE, svg.STEP_PROFILE]
     for t in range(4):
         out = layer(t, *args)
@@ -382,7 +382,7 @@ def test_layer_schedule_dense_then_profiled_then_reused():
 
 # ------------------------------------------- five-pass step building blocks
 
-@pytest.mark.parametrize("key", ["cfg0", "ragged128", "smallS", "oddsplit", "cfg2"])
+@pytest.mark.parametrize("key", ["tiny", "ragged128", "smallS", "oddsplit", "wan"])
 def test_selective_norm_passes_match_the_two_stage_path(key):
     """K alone, and {raw Q normalised + K, V moved} in one pass, give the same
     bits as normalising both and then moving all three."""
@@ -402,7 +402,7 @@ def test_selective_norm_passes_match_the_two_stage_path(key):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
-@pytest.mark.parametrize("key", ["cfg0", "ragged128", "smallS128", "oddsplit", "cfg2"])
+@pytest.mark.parametrize("key", ["tiny", "ragged128", "smallS128", "oddsplit", "wan"])
 def test_profile_raw_q_equals_profile_on_normalised_q(key):
     """The sampled rows normalised inside the profiling kernel are the rows the
     norm pass writes, so kinds and MSEs agree bit for bit."""

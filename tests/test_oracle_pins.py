@@ -212,7 +212,7 @@ def test_hunyuan_spatial_density_golden():
     """The HunyuanVideo 720p workload states about 9 % key density for a
     +-1-frame spatial window; exact counts from the oracle's mask."""
     g = json.load(open(os.path.join(GOLDEN, "density.json")))
-    wl = W.CONFIGS[3]
+    wl = W.HUNYUAN
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
     z = np.zeros((1, 1, wl.L, wl.d), np.uint16)
     sh1 = oracle.make_shape(1, 1, wl.d, wl.F, wl.Hs, wl.Ws, wl.T)
@@ -231,7 +231,7 @@ def test_hunyuan_spatial_density_golden():
 
 def test_profile_sample_fraction_golden():
     g = json.load(open(os.path.join(GOLDEN, "profiling_sample.json")))
-    wl = W.CONFIGS[3]
+    wl = W.HUNYUAN
     frac = wl.n_samples / wl.L
     assert wl.n_samples == g["n_queries"]
     assert abs(frac - g["fraction"]) < g["tolerance"]
@@ -336,8 +336,8 @@ def test_layout_roundtrip_and_fixed_points():
 
 # ------------------------------------------------------------ profiling ----
 
-def test_profile_brute_force_config0():
-    wl = W.CONFIGS[0]
+def test_profile_brute_force_tiny():
+    wl = W.TINY
     inp = W.make_inputs(wl)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
     qn = oracle.qknorm_rope(sh, pr, inp["q"], inp["gamma_q"])
@@ -370,8 +370,8 @@ def test_profile_classifies_strongly_planted_heads():
     assert list(choice) == [0, 1, 1, 0]
 
 
-def test_profile_planted_config2():
-    wl = W.CONFIGS[2]
+def test_profile_planted_wan():
+    wl = W.WAN
     inp = W.make_inputs(wl)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
     qn = oracle.qknorm_rope(sh, pr, inp["q"], inp["gamma_q"])
@@ -412,9 +412,8 @@ def _closed_form_tiles(wl, kind, w, r):
     return listed, full
 
 
-@pytest.mark.parametrize("cfg", [0, 1])
-def test_block_list_brute_force_equals_interval_form(cfg):
-    wl = W.CONFIGS[cfg]
+@pytest.mark.parametrize("wl", [W.TINY, W.COGVIDEOX], ids=["tiny", "cogvideox"])
+def test_block_list_brute_force_equals_interval_form(wl):
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
     kinds = np.array([W.SPATIAL, W.TEMPORAL, W.DENSE] * (wl.H // 2 + 1), np.uint8)[:wl.H]
     row_ptr, col, full = oracle.block_list(sh, pr, kinds)

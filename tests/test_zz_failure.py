@@ -26,7 +26,7 @@ def test_bounded_wait_times_out_and_the_context_survives():
     assert time.time() - t0 < 30
     svg.sync_status()                                   # the error word was cleared
     # the same context still runs a whole step correctly
-    wl = W.CONFIGS[0]
+    wl = W.TINY
     inp = W.make_inputs(wl)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
     pb = svg.Problem.from_workload(wl)

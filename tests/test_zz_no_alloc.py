@@ -31,9 +31,9 @@ def _inputs(wl):
     return pb, qn, kn, dev(inp["v"]), dev(inp["sample_idx"])
 
 
-@pytest.mark.parametrize("cfg", [0, 2])
-def test_noalloc_matches_workspace_entry_point_twice(cfg):
-    pb, qn, kn, v, si = _inputs(W.CONFIGS[cfg])
+@pytest.mark.parametrize("wl", [W.TINY, W.WAN], ids=["tiny", "wan"])
+def test_noalloc_matches_workspace_entry_point_twice(wl):
+    pb, qn, kn, v, si = _inputs(wl)
     kinds_ref, mse_ref = svg.profile_heads(pb, qn, kn, v, si)
     svg.sync_status()
     kinds_ref, mse_ref = kinds_ref.cpu().numpy(), mse_ref.cpu().numpy().astype(np.float64)
