@@ -37,6 +37,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "svg_oracle.c")
+_SRC2 = os.path.join(_HERE, "svg2_oracle.c")
 _BUILD = os.path.join(_HERE, "_build")
 _LIB = os.path.join(_BUILD, "liboracle.so")
 _lock = threading.Lock()
@@ -60,10 +61,12 @@ class OraParams(ctypes.Structure):
 def build(force: bool = False) -> str:
     """Compile svg_oracle.c into oracle/_build/liboracle.so (gcc, -O2, OpenMP)."""
     os.makedirs(_BUILD, exist_ok=True)
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC2))
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
         tmp = _LIB + f".tmp{os.getpid()}"
+        # -std=c11 keeps a*b+c unfused (no contraction), as the oracle's text says
         subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-                               "-o", tmp, _SRC, "-lm"])
+                               "-o", tmp, _SRC, _SRC2, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -94,6 +97,17 @@ def lib():
             L.ora_profile.argtypes = [sh, pr, vp, vp, vp, ctypes.c_int, vp, vp, vp]
             L.ora_block_list.restype = i64
             L.ora_block_list.argtypes = [sh, pr, vp, vp, vp, vp]
+            ci = ctypes.c_int
+            L.ora2_kmeans_init.argtypes = [vp, ci, i64, i64, ci, ci, vp]
+            L.ora2_assign.argtypes = [vp, ci, i64, i64, ci, ci, vp, vp]
+            L.ora2_update.argtypes = [vp, ci, i64, i64, ci, ci, vp, vp, vp]
+            L.ora2_kmeans.argtypes = [vp, ci, i64, i64, ci, ci, ci, vp, vp, vp]
+            L.ora2_permutation.argtypes = [vp, ci, i64, ci, vp, vp]
+            L.ora2_select.argtypes = [vp, vp, vp, ci, ci, ci, ci, ctypes.c_double, ctypes.c_double, vp, vp]
+            L.ora2_attention_rows.argtypes = [ci, i64, i64, ci, ci, ci, ctypes.c_double, vp, vp, vp, vp, vp, vp,
+                                              i64, vp, vp, vp]
+            L.ora2_block_list.restype = i64
+            L.ora2_block_list.argtypes = [ci, i64, i64, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp, vp, i64]
             _lib = L
     return _lib
 
@@ -251,3 +265,102 @@ def step(wl, inputs, kinds=None):
     if kinds is None:
         mse, kinds = profile(sh, pr, qn, kn, inputs["v"], inputs["sample_idx"])
     return {"qn": qn, "kn": kn, "mse": mse, "kinds": np.asarray(kinds, np.uint8)}
+
+
+# ------------------------------------------------ semantic-aware permutation --
+# "Sparse VideoGen2" explainer, "A. 语义感知排列" and "B. 基于质心的 Top-p 选择";
+# the readings are stated at the top of svg2_oracle.c.
+
+def kmeans_init(x, Lv: int, C: int) -> np.ndarray:
+    """Centroid c = video row floor(c*Lv/C) of each head; x bf16 [B,H,L,d] -> float32 [BH,C,d]."""
+    x = _c(x, np.uint16)
+    BH, L, d = x.shape[0] * x.shape[1], x.shape[2], x.shape[3]
+    cent = np.empty((BH, C, d), np.float32)
+    lib().ora2_kmeans_init(_ptr(x), BH, L, Lv, d, C, _ptr(cent))
+    return cent
+
+
+def kmeans_assign(x, Lv: int, cent) -> np.ndarray:
+    x = _c(x, np.uint16)
+    cent = _c(cent, np.float32)
+    BH, L, d = x.shape[0] * x.shape[1], x.shape[2], x.shape[3]
+    out = np.empty((BH, Lv), np.uint8)
+    lib().ora2_assign(_ptr(x), BH, L, Lv, d, cent.shape[1], _ptr(cent), _ptr(out))
+    return out
+
+
+def kmeans_update(x, Lv: int, assign, cent):
+    """Returns (new centroids float32 [BH,C,d], counts int32 [BH,C]); `cent` is not modified."""
+    x = _c(x, np.uint16)
+    cent = np.array(cent, dtype=np.float32, copy=True)
+    assign = _c(assign, np.uint8)
+    BH, L, d = x.shape[0] * x.shape[1], x.shape[2], x.shape[3]
+    counts = np.empty((BH, cent.shape[1]), np.int32)
+    lib().ora2_update(_ptr(x), BH, L, Lv, d, cent.shape[1], _ptr(assign), _ptr(cent), _ptr(counts))
+    return cent, counts
+
+
+def kmeans(x, Lv: int, C: int, iters: int, cent=None):
+    """`iters` Lloyd rounds from `cent` (default: kmeans_init) and a final
+    assignment.  Returns (centroids, assign uint8 [BH,Lv], counts int32 [BH,C])."""
+    x = _c(x, np.uint16)
+    BH, L, d = x.shape[0] * x.shape[1], x.shape[2], x.shape[3]
+    cent = kmeans_init(x, Lv, C) if cent is None else np.array(cent, dtype=np.float32, copy=True)
+    assign = np.empty((BH, Lv), np.uint8)
+    counts = np.empty((BH, C), np.int32)
+    lib().ora2_kmeans(_ptr(x), BH, L, Lv, d, C, iters, _ptr(cent), _ptr(assign), _ptr(counts))
+    return cent, assign, counts
+
+
+def cluster_permutation(assign, C: int):
+    """Stable counting sort: (perm int32 [BH,Lv] position -> row, off int32 [BH,C+1])."""
+    assign = _c(assign, np.uint8)
+    BH, Lv = assign.shape
+    perm_ = np.empty((BH, Lv), np.int32)
+    off = np.empty((BH, C + 1), np.int32)
+    lib().ora2_permutation(_ptr(assign), BH, Lv, C, _ptr(perm_), _ptr(off))
+    return perm_, off
+
+
+def select_top_p(cq, ck, nk, scale: float, p: float, want_weight=False):
+    """Top-p key clusters per query cluster: sel uint64 [BH,Cq] (and weights [BH,Cq,Ck])."""
+    cq, ck = _c(cq, np.float32), _c(ck, np.float32)
+    nk = _c(nk, np.int32)
+    BH, Cq, d = cq.shape
+    Ck = ck.shape[1]
+    sel = np.empty((BH, Cq), np.uint64)
+    w = np.empty((BH, Cq, Ck), np.float64) if want_weight else None
+    lib().ora2_select(_ptr(cq), _ptr(ck), _ptr(nk), BH, Cq, Ck, d, float(scale), float(p), _ptr(sel), _ptr(w))
+    return (sel, w) if want_weight else sel
+
+
+def attention2_rows(q, k, v, Lv: int, aq, ak, sel, rows, scale=None, want_lse=False):
+    """fp64 attention with the cluster mask, model order; rows = bh*L + token."""
+    q, k, v = (_c(t, np.uint16) for t in (q, k, v))
+    aq, ak = _c(aq, np.uint8), _c(ak, np.uint8)
+    sel = _c(sel, np.uint64)
+    rows = _c(rows, np.int64)
+    BH, L, d = q.shape[0] * q.shape[1], q.shape[2], q.shape[3]
+    sc = 1.0 / np.sqrt(d) if scale is None else scale
+    out = np.empty((len(rows), d), np.float64)
+    lse = np.empty(len(rows), np.float64) if want_lse else None
+    lib().ora2_attention_rows(BH, L, Lv, d, sel.shape[1], 0, sc, _ptr(q), _ptr(k), _ptr(v), _ptr(aq), _ptr(ak),
+                              _ptr(sel), len(rows), _ptr(rows), _ptr(out), _ptr(lse))
+    return (out, lse) if want_lse else out
+
+
+def block_list2(L: int, Lv: int, bq: int, bk: int, aq, ak, perm_q, perm_k, sel):
+    """Tile list over the permuted order by brute force: (row_ptr, col, full)."""
+    aq, ak = _c(aq, np.uint8), _c(ak, np.uint8)
+    perm_q, perm_k = _c(perm_q, np.int32), _c(perm_k, np.int32)
+    sel = _c(sel, np.uint64)
+    BH = aq.shape[0]
+    nqb, nkb = -(-L // bq), -(-L // bk)
+    cap = BH * nqb * nkb
+    row_ptr = np.empty(BH * nqb + 1, np.int32)
+    col = np.empty(cap, np.int32)
+    full = np.empty(cap, np.uint8)
+    n = lib().ora2_block_list(BH, L, Lv, sel.shape[1], 0, bq, bk, _ptr(aq), _ptr(ak), _ptr(perm_q), _ptr(perm_k),
+                              _ptr(sel), _ptr(row_ptr), _ptr(col), _ptr(full), cap)
+    return row_ptr, col[:n], full[:n]
+
