@@ -363,6 +363,96 @@ def run_gpu(args, rank, world, local_rank):
     return line
 
 
+# ------------------------------------- semantic-aware permutation (SVG2) --
+
+def run_svg2(args):
+    """The SVG2 step ("Sparse VideoGen2" explainer, "A. 语义感知排列", "B. 基于质心的
+    Top-p 选择") on one GPU: QK-Norm + RoPE of Q and K, k-means of Q and K
+    (warm-started from the previous step's centroids), cluster sort, top-p key
+    clusters, permutation of Q, K, V, block index, attention written back in
+    model order.  Prints one JSON line; not the default bench line."""
+    import torch
+
+    import sparse_attention_video_qk_b200 as svg
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    wl = W.WORKLOADS[args.workload]
+    pb = svg.Problem.from_workload(wl)
+    inp = W.make_inputs(wl)
+    q, k, v = (torch.from_numpy(inp[n]).view(torch.bfloat16).to(device) for n in ("q", "k", "v"))
+    gq, gk = (torch.from_numpy(inp[n]).to(device) for n in ("gamma_q", "gamma_k"))
+    table = torch.from_numpy(svg.rope_table(pb)).to(device)
+    Cq, Ck, iters, top_p = args.svg2_clusters, args.svg2_clusters, args.svg2_iters, args.svg2_top_p
+    stream = torch.cuda.current_stream()
+    st = {}
+
+    def step(ev=None):
+        mark = (lambda i: ev[i].record(stream)) if ev is not None else (lambda i: None)
+        mark(0)
+        qn, kn = svg.qknorm_rope(pb, q, k, gq, gk, table)
+        mark(1)
+        cq, aq, nq = svg.svg2_kmeans(pb, qn, Cq, iters, st.get("cq"))
+        ck, ak, nk = svg.svg2_kmeans(pb, kn, Ck, iters, st.get("ck"))
+        st["cq"], st["ck"] = cq, ck
+        mark(2)
+        pq, qoff = svg.svg2_permutation(pb, aq, Cq)
+        pk, koff = svg.svg2_permutation(pb, ak, Ck)
+        sel = svg.svg2_select(pb, cq, ck, nk, top_p)
+        mark(3)
+        qp, kp, vp = svg.svg2_permute(pb, pq, pk, qn, kn, v)
+        mark(4)
+        rp, col, full = svg.svg2_block_index(pb, qoff, koff, sel)
+        mark(5)
+        out = svg.svg2_attention(pb, qp, kp, vp, qoff, koff, sel, pq, rp, col, full)
+        mark(6)
+        st.update(rp=rp, col=col, sel=sel, out=out)
+
+    names = ("qk_norm_rope", "kmeans_q_k", "sort_select", "permute", "block_index", "attention")
+    for _ in range(args.warmup):
+        step()
+    svg.sync_status()
+    n_ent = int(st["rp"][-1])
+    flops = kept_tile_flops(st["rp"].cpu().numpy(), st["col"][:n_ent].cpu().numpy(), wl)
+    sel_bits = np.array([bin(int(x)).count("1") for x in st["sel"].cpu().numpy().view(np.uint64).ravel()])
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        clk.start()
+        for s in range(args.steps):
+            step(ev[s])
+        torch.cuda.synchronize()
+        clk.stop()
+    svg.sync_status()
+    stage_ms = {n: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps))
+                for i, n in enumerate(names)}
+    ms = statistics.mean(ev[s][0].elapsed_time(ev[s][-1]) for s in range(args.steps))
+    pk, pk_src = peaks()
+    attn_tflops = flops / (stage_ms["attention"] * 1e-3) / 1e12
+    BH, Lv, d = wl.B * wl.H, wl.Lv, wl.d
+    # one assignment pass: Lv*C*d (subtract, multiply-add) pairs per head and tensor
+    assign_pairs = 2.0 * BH * Lv * Cq * d * (iters + 1)
+    line = {
+        "metric": "SVG2 layer ms and effective TFLOP/s over kept tiles",
+        "value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V with planted spatial/temporal heads; no model weights)",
+        "config": {"workload": f"{wl.name} ({SHAPE_LABEL[wl.name]}), semantic-aware permutation",
+                   "clusters_q": Cq, "clusters_k": Ck, "kmeans_iters": iters, "top_p": top_p,
+                   "kept_tile_tflop": round(flops / 1e12, 4),
+                   "tile_density": round(n_ent / (BH * wl.nqb * wl.nkb), 4),
+                   "mean_key_clusters_selected": round(float(sel_bits.mean()), 2)},
+        "stage_ms": {n: round(t, 4) for n, t in stage_ms.items()},
+        "kmeans_pair_rate_g_per_s": round(assign_pairs / (stage_ms["kmeans_q_k"] * 1e-3) / 1e9, 1),
+        "roofline": {"kernel": f"attn2_kernel<{d}> (svg2_attention)", "bound": "tensor",
+                     "achieved": round(attn_tflops, 2), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": round(attn_tflops / pk["bf16_tflops_sustained"], 4),
+                     "peak_source": f"{pk_src} bf16 sustained", "traffic": None},
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------ sparsity sweep --
 
 def token_density(wl, kind):
@@ -554,6 +644,11 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=960)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--svg2", action="store_true",
+                    help="time the semantic-aware permutation step (SVG2) instead of the default step")
+    ap.add_argument("--svg2-clusters", type=int, default=64)
+    ap.add_argument("--svg2-iters", type=int, default=2)
+    ap.add_argument("--svg2-top-p", type=float, default=0.9)
     ap.add_argument("--sweep", action="store_true",
                     help="forced-kind sparsity sweep (one GPU); prints one JSON line with every point")
     args = ap.parse_args()
@@ -564,6 +659,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if world != args.gpus:
         world = max(world, 1)
+    if args.svg2:
+        if rank == 0:
+            run_svg2(args)
+        return
     if args.sweep:
         if rank == 0:
             print(json.dumps(run_sweep(args)), flush=True)

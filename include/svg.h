@@ -245,6 +245,71 @@ svg_status svg_attention_step(const svg_shape* shape, const svg_params* params,
                               int32_t* row_ptr, int32_t* col, uint8_t* full, int64_t capacity,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------ semantic-aware permutation ("Sparse VideoGen2") */
+/* The second workload ("Sparse VideoGen2" explainer, "A. 语义感知排列" and
+ * "B. 基于质心的 Top-p 选择"): per head, the video rows of Q and of K are
+ * clustered by k-means, each tensor is sorted so that every cluster is
+ * contiguous, every query cluster attends the top-p key clusters estimated
+ * from size-weighted centroid scores, and text tokens stay at the end, kept by
+ * every query and keeping every key.  Cluster counts are 1..64 (a query
+ * cluster's key set is one 64-bit mask).  Decisions taken from floating point
+ * follow a fixed operation order (stated with each call), so they do not
+ * depend on scheduling. */
+
+/* Bytes of device scratch svg2_kmeans needs: B*H*C*d*8. */
+size_t svg2_kmeans_workspace_size(const svg_shape* shape, int C);
+
+/* k-means of the F*Hs*Ws video rows of every head of x (device bf16 [B,H,L,d]):
+ * with init != 0 the centroids start at video rows floor(c*Lv/C); otherwise
+ * `cent` holds the starting centroids (e.g. the previous denoising step's: the
+ * pages' centroid cache).  `iters` rounds of (assign every row to its nearest
+ * centroid; move each centroid to the mean of its rows, an empty cluster keeps
+ * its centroid), then a final assignment.  Distance sum_i (x_i - c_i)^2 in float
+ * with fused multiply-add in the order i = 0..d-1, the lowest index on a tie;
+ * sums in 64-bit fixed point (x * 2^40 truncated), mean ((double)sum / 2^40) /
+ * count rounded to float.
+ * cent: device float [B*H][C][d] (in/out); assign: device uint8 [B*H][Lv];
+ * counts: device int32 [B*H][C], the sizes of the final assignment. */
+svg_status svg2_kmeans(const svg_shape* shape, const uint16_t* x, int C, int iters, int init, float* cent,
+                       uint8_t* assign, int32_t* counts, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Stable counting sort of each head's video rows by cluster: perm (device int32
+ * [B*H][Lv]) = the row placed at each position, off (device int32 [B*H][C+1]) =
+ * the first position of each cluster (off[C] = Lv). */
+svg_status svg2_permutation(const svg_shape* shape, const uint8_t* assign, int C, int32_t* perm, int32_t* off,
+                            void* stream);
+
+/* Top-p key clusters of every query cluster: s_ij = scale * (cq_i . ck_j) in
+ * double (multiply and add in the order of the d components), weights
+ * w_ij = n_j * exp(s_ij - max over non-empty j), key clusters in decreasing
+ * weight (lower index first on a tie), and the shortest prefix whose running sum
+ * reaches top_p times the sum of all weights (summed in index order).
+ * cq, ck: device float [B*H][Cq|Ck][d]; counts_k: device int32 [B*H][Ck];
+ * sel: device uint64 [B*H][Cq], bit j = key cluster j.  scale = softmax_scale or
+ * 1/sqrt(d) in double.  0 < top_p <= 1. */
+svg_status svg2_select(const svg_shape* shape, const svg_params* params, const float* cq, const float* ck,
+                       const int32_t* counts_k, int Cq, int Ck, double top_p, uint64_t* sel, void* stream);
+
+/* Q, K, V into cluster order: video position p of q_out takes row perm_q[p];
+ * k_out and v_out take row perm_k[p]; text rows are copied in place. */
+svg_status svg2_permute(const svg_shape* shape, const int32_t* perm_q, const int32_t* perm_k, const uint16_t* q,
+                        const uint16_t* k, const uint16_t* v, uint16_t* q_out, uint16_t* k_out, uint16_t* v_out,
+                        void* stream);
+
+/* Block index over the cluster order (same CSR format and `full` meaning as
+ * svg_build_block_index): tile (qb, kb) is listed iff one of its pairs is kept. */
+svg_status svg2_build_block_index(const svg_shape* shape, const svg_params* params, int Cq, int Ck,
+                                  const int32_t* qoff, const int32_t* koff, const uint64_t* sel, int32_t* row_ptr,
+                                  int32_t* col, uint8_t* full, int64_t capacity, void* stream);
+
+/* Block-sparse attention in cluster order (q, k, v from svg2_permute) with the
+ * cluster mask, written back in model order: video position p goes to row
+ * perm_q[p] of out (and of lse_out, if given).  Requires block_q = 128. */
+svg_status svg2_attention(const svg_shape* shape, const svg_params* params, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, int Cq, int Ck, const int32_t* qoff, const int32_t* koff,
+                          const uint64_t* sel, const int32_t* perm_q, const int32_t* row_ptr, const int32_t* col,
+                          const uint8_t* full, uint16_t* out, float* lse_out, void* stream);
+
 /* ----------------------------------------------------------- host helpers */
 
 /* n distinct video-token indices in [0, Lv) into host_out[0..n): the first n slots of

@@ -364,3 +364,16 @@ def block_list2(L: int, Lv: int, bq: int, bk: int, aq, ak, perm_q, perm_k, sel):
                               _ptr(sel), _ptr(row_ptr), _ptr(col), _ptr(full), cap)
     return row_ptr, col[:n], full[:n]
 
+
+
+def permute_rows(x, Lv: int, perm):
+    """Video position p of every head takes row perm[bh, p]; text rows stay
+    (the cluster-contiguous order of step 2).  x bf16 [B,H,L,d]."""
+    x = _c(x, np.uint16)
+    B, H, L, d = x.shape
+    perm = _c(perm, np.int32).reshape(B, H, Lv)
+    out = x.copy()
+    for b in range(B):
+        for h in range(H):
+            out[b, h, :Lv] = x[b, h, perm[b, h]]
+    return out

@@ -51,6 +51,14 @@ SIGNATURES = {
                                   _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
                                   _vp, _sz, _vp]),
     "svg_sample_queries": (_i32, [ctypes.c_uint64, _i64, _i32, _vp]),
+    "svg2_kmeans_workspace_size": (_sz, [_SP, _i32]),
+    "svg2_kmeans": (_i32, [_SP, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "svg2_permutation": (_i32, [_SP, _vp, _i32, _vp, _vp, _vp]),
+    "svg2_select": (_i32, [_SP, _PP, _vp, _vp, _vp, _i32, _i32, ctypes.c_double, _vp, _vp]),
+    "svg2_permute": (_i32, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "svg2_build_block_index": (_i32, [_SP, _PP, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp]),
+    "svg2_attention": (_i32, [_SP, _PP, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                              _vp]),
     "svg_step_policy": (_i32, [_i32, _i32, ctypes.c_float, _i32, ctypes.POINTER(ctypes.c_int)]),
     "svg_rope_table_size": (_sz, [_SP, _PP]),
     "svg_rope_table_fill": (_i32, [_SP, _PP, _vp]),

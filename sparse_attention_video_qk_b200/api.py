@@ -375,6 +375,110 @@ def sparse_attention(pb: Problem, q_host, k_host, v_host, gamma_q, gamma_k, samp
     return pipeline(q_host, k_host, v_host, gamma_q, gamma_k, sample_idx, out_host)
 
 
+# ------------------------------------------- semantic-aware permutation --
+
+def svg2_kmeans(pb: Problem, x, C: int, iters: int, cent=None, stream=None):
+    """k-means of the video rows of every head of x (bf16 [B,H,L,d]); starts from
+    `cent` (float [B*H, C, d], e.g. the previous step's) or from evenly spaced
+    rows.  Returns (cent, assign uint8 [B*H, Lv], counts int32 [B*H, C])."""
+    sh = pb.c_shape()
+    bh, dev = pb.B * pb.H, x.device
+    init = cent is None
+    if init:
+        cent = torch.empty(bh, C, pb.d, dtype=torch.float32, device=dev)
+    assign = torch.empty(bh, pb.Lv, dtype=torch.uint8, device=dev)
+    counts = torch.empty(bh, C, dtype=torch.int32, device=dev)
+    ws = torch.empty(max(lib().svg2_kmeans_workspace_size(ctypes.byref(sh), C), 16), dtype=torch.uint8, device=dev)
+    check(lib().svg2_kmeans(ctypes.byref(sh), _p(x), C, iters, int(init), _p(cent), _p(assign), _p(counts), _p(ws),
+                            ws.numel(), _stream(stream)), "svg2_kmeans")
+    return cent, assign, counts
+
+
+def svg2_permutation(pb: Problem, assign, C: int, stream=None):
+    """Stable cluster sort: (perm int32 [B*H, Lv], off int32 [B*H, C+1])."""
+    sh = pb.c_shape()
+    bh = pb.B * pb.H
+    perm = torch.empty(bh, pb.Lv, dtype=torch.int32, device=assign.device)
+    off = torch.empty(bh, C + 1, dtype=torch.int32, device=assign.device)
+    check(lib().svg2_permutation(ctypes.byref(sh), _p(assign), C, _p(perm), _p(off), _stream(stream)),
+          "svg2_permutation")
+    return perm, off
+
+
+def svg2_select(pb: Problem, cq, ck, counts_k, top_p: float, stream=None):
+    """Top-p key clusters per query cluster: uint64 masks [B*H, Cq] (as int64)."""
+    sh, pr = pb.c_shape(), pb.c_params()
+    bh, Cq, Ck = pb.B * pb.H, cq.shape[1], ck.shape[1]
+    sel = torch.empty(bh, Cq, dtype=torch.int64, device=cq.device)
+    check(lib().svg2_select(ctypes.byref(sh), ctypes.byref(pr), _p(cq), _p(ck), _p(counts_k), Cq, Ck, float(top_p),
+                            _p(sel), _stream(stream)), "svg2_select")
+    return sel
+
+
+def svg2_permute(pb: Problem, perm_q, perm_k, q, k, v, stream=None):
+    sh = pb.c_shape()
+    qo, ko, vo = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    check(lib().svg2_permute(ctypes.byref(sh), _p(perm_q), _p(perm_k), _p(q), _p(k), _p(v), _p(qo), _p(ko), _p(vo),
+                             _stream(stream)), "svg2_permute")
+    return qo, ko, vo
+
+
+def svg2_block_index(pb: Problem, qoff, koff, sel, capacity=None, stream=None):
+    sh, pr = pb.c_shape(), pb.c_params()
+    Cq, Ck = qoff.shape[1] - 1, koff.shape[1] - 1
+    if capacity is None:
+        capacity = block_index_capacity(pb)
+    dev = qoff.device
+    row_ptr = torch.empty(pb.B * pb.H * pb.nqb + 1, dtype=torch.int32, device=dev)
+    col = torch.empty(capacity, dtype=torch.int32, device=dev)
+    full = torch.empty(capacity, dtype=torch.uint8, device=dev)
+    check(lib().svg2_build_block_index(ctypes.byref(sh), ctypes.byref(pr), Cq, Ck, _p(qoff), _p(koff), _p(sel),
+                                       _p(row_ptr), _p(col), _p(full), capacity, _stream(stream)),
+          "svg2_build_block_index")
+    return row_ptr, col, full
+
+
+def svg2_attention(pb: Problem, q, k, v, qoff, koff, sel, perm_q, row_ptr, col, full, out=None, want_lse=False,
+                   stream=None):
+    """Attention in cluster order, written back in model order."""
+    sh, pr = pb.c_shape(), pb.c_params()
+    Cq, Ck = qoff.shape[1] - 1, koff.shape[1] - 1
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty(pb.B, pb.H, pb.L, dtype=torch.float32, device=q.device) if want_lse else None
+    check(lib().svg2_attention(ctypes.byref(sh), ctypes.byref(pr), _p(q), _p(k), _p(v), Cq, Ck, _p(qoff), _p(koff),
+                               _p(sel), _p(perm_q), _p(row_ptr), _p(col), _p(full), _p(out), _p(lse),
+                               _stream(stream)), "svg2_attention")
+    return (out, lse) if want_lse else out
+
+
+class SVG2Layer:
+    """The semantic-aware permutation step on normalised Q, K and V: k-means of
+    Q and K (warm-started from the previous call's centroids, the pages'
+    centroid cache), cluster sort, top-p key clusters, block index, attention
+    in cluster order written back in model order."""
+
+    def __init__(self, pb: Problem, Cq: int = 64, Ck: int = 64, iters: int = 2, top_p: float = 0.9):
+        self.pb, self.Cq, self.Ck, self.iters, self.top_p = pb, Cq, Ck, iters, top_p
+        self.cq = self.ck = None
+        self.last = None
+
+    def __call__(self, qn, kn, v, stream=None):
+        pb = self.pb
+        cq, aq, nq = svg2_kmeans(pb, qn, self.Cq, self.iters, self.cq, stream)
+        ck, ak, nk = svg2_kmeans(pb, kn, self.Ck, self.iters, self.ck, stream)
+        self.cq, self.ck = cq, ck
+        pq, qoff = svg2_permutation(pb, aq, self.Cq, stream)
+        pk, koff = svg2_permutation(pb, ak, self.Ck, stream)
+        sel = svg2_select(pb, cq, ck, nk, self.top_p, stream)
+        qp, kp, vp = svg2_permute(pb, pq, pk, qn, kn, v, stream)
+        row_ptr, col, full = svg2_block_index(pb, qoff, koff, sel, stream=stream)
+        out = svg2_attention(pb, qp, kp, vp, qoff, koff, sel, pq, row_ptr, col, full, stream=stream)
+        self.last = dict(assign_q=aq, assign_k=ak, counts_q=nq, counts_k=nk, perm_q=pq, perm_k=pk, qoff=qoff,
+                         koff=koff, sel=sel, row_ptr=row_ptr, col=col, full=full)
+        return out
+
+
 # ------------------------------------------------------ denoising schedule --
 
 STEP_DENSE, STEP_PROFILE, STEP_REUSE = C.SVG_STEP_DENSE, C.SVG_STEP_PROFILE, C.SVG_STEP_REUSE

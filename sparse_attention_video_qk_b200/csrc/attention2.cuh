@@ -271,9 +271,18 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
     const int q4 = warp & 3;                       // TMEM lane quarter
     const int r = q4 * 32 + lane;
     const int row = (qb0 + w) * g.bq + r;
-    const int kind = a.kind[bh];
+    const int kind = a.sel ? static_cast<int>(SVG_HEAD_DENSE) : a.kind[bh];
     int lo, hi;
     row_interval(g, kind, row, lo, hi);
+    // semantic-permutation mask: this row's key-cluster set (text rows: all)
+    uint64_t rmask = ~0ull;
+    const int32_t* ko = nullptr;
+    if (a.sel) {
+      ko = a.koff + static_cast<int64_t>(bh) * (a.Ck + 1);
+      if (row < g.Lv)
+        rmask = a.sel[static_cast<int64_t>(bh) * a.Cq + cluster_of(a.qoff + static_cast<int64_t>(bh) * (a.Cq + 1),
+                                                                    a.Cq, row)];
+    }
     const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const uint32_t tS = tl + C::tm_s(w), tO = tl + C::tm_o(w);
     const float sl2 = a.scale_log2;
@@ -317,12 +326,29 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
           for (int c = 0; c < 32; c++) v[c] = __float_as_uint(-INFINITY);
         } else if (mode[h] == 1) {
           const int k0 = kbs[h] * 64 + (q & 1) * 32;
+          if (ko) {
+            // key clusters are contiguous: walk their boundaries along the 32 columns
+            int jc = (k0 < g.Lv) ? cluster_of(ko, a.Ck, k0) : 0;
+            int next = ko[jc + 1];
+            for (int c = 0; c < 32; c++) {
+              const int kk = k0 + c;
+              bool keep;
+              if (kk >= g.Lv) {
+                keep = kk < g.L;
+              } else {
+                while (kk >= next) next = ko[++jc + 1];
+                keep = (rmask >> jc) & 1ull;
+              }
+              if (!keep) v[c] = __float_as_uint(-INFINITY);
+            }
+          } else {
 #pragma unroll
-          for (int c = 0; c < 32; c++) {
-            const int kk = k0 + c;
-            const bool keep = (static_cast<unsigned>(kk - lo) < static_cast<unsigned>(hi - lo)) ||
-                              (static_cast<unsigned>(kk - g.Lv) < static_cast<unsigned>(g.T));
-            if (!keep) v[c] = __float_as_uint(-INFINITY);
+            for (int c = 0; c < 32; c++) {
+              const int kk = k0 + c;
+              const bool keep = (static_cast<unsigned>(kk - lo) < static_cast<unsigned>(hi - lo)) ||
+                                (static_cast<unsigned>(kk - g.Lv) < static_cast<unsigned>(g.T));
+              if (!keep) v[c] = __float_as_uint(-INFINITY);
+            }
           }
         }
       };
@@ -440,7 +466,7 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
     if (ok && nT > 0 && __all_sync(0xffffffffu, mbar_wait(b_o(w), (nT - 1) & 1, abort_flag))) {
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row(g, a.model_order, kind, row);
+      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row(a, kind, bh, row);
       uint16_t* orow = a.out + orow_i * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; c++) {
@@ -462,7 +488,7 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
       }
       if (row_ok && a.lse) a.lse[orow_i] = (l > 0.f) ? (m_use * 0.69314718055994531f + logf(l)) : -INFINITY;
     } else if (ok && nT == 0 && row_ok) {
-      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row(g, a.model_order, kind, row);
+      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row(a, kind, bh, row);
       uint4* dst = reinterpret_cast<uint4*>(a.out + orow_i * D);
       for (int v = 0; v < D / 8; v++) dst[v] = make_uint4(0, 0, 0, 0);
       if (a.lse) a.lse[orow_i] = -INFINITY;

@@ -50,6 +50,18 @@ __device__ __forceinline__ void row_interval(const Geometry& g, int kind, int ro
   }
 }
 
+// Cluster of position p in a cluster-sorted order: the c with off[c] <= p <
+// off[c+1] (empty clusters, off[c] == off[c+1], are skipped).
+__device__ __forceinline__ int cluster_of(const int32_t* off, int C, int p) {
+  int lo = 0, hi = C - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= p) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
 __device__ __forceinline__ bool key_kept(const Geometry& g, int lo, int hi, int k) {
   return (k >= lo && k < hi) || (k >= g.Lv && k < g.L);
 }

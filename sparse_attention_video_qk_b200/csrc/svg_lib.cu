@@ -7,12 +7,14 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "attention.cuh"
 #include "attention2.cuh"
 #include "block_index.cuh"
 #include "profile_tc.cuh"
 #include "rowmap.cuh"
+#include "svg2.cuh"
 #include "svg_common.cuh"
 
 using namespace svg;
@@ -484,14 +486,17 @@ svg_status svg_build_block_index(const svg_shape* s, const svg_params* p, const 
 
 // Block-sparse attention; model_order = 1 also applies the inverse layout
 // (temporal heads' rows are stored back in frame-major order).
+// `cluster` (or null) carries the semantic-permutation mask fields (sel, qoff,
+// koff, Cq, Ck, out_perm); head_kind is then unused.
 static svg_status attention_launch(const svg_shape* s, const svg_params* p, const uint16_t* q, const uint16_t* k,
                                    const uint16_t* v, const uint8_t* head_kind, const int32_t* row_ptr,
                                    const int32_t* col, const uint8_t* full, uint16_t* out, float* lse_out,
-                                   int model_order, void* stream) {
+                                   int model_order, void* stream, const AttnArgs* cluster = nullptr) {
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if ((st = check_params(s, p, true)) != SVG_OK) return st;
-  if (!q || !k || !v || !head_kind || !row_ptr || !col || !full || !out) return SVG_ERR_INVALID_ARG;
+  if (!q || !k || !v || (!head_kind && !cluster) || !row_ptr || !col || !full || !out) return SVG_ERR_INVALID_ARG;
+  if (cluster && p->block_q != 128) return SVG_ERR_UNSUPPORTED;
   const void* ptrs[] = {q, k, v, out};
   for (const void* ptr : ptrs)
     if (!aligned16(ptr)) return SVG_ERR_ALIGNMENT;
@@ -506,6 +511,14 @@ static svg_status attention_launch(const svg_shape* s, const svg_params* p, cons
   a.out = out;
   a.lse = lse_out;
   a.model_order = model_order;
+  if (cluster) {
+    a.sel = cluster->sel;
+    a.qoff = cluster->qoff;
+    a.koff = cluster->koff;
+    a.Cq = cluster->Cq;
+    a.Ck = cluster->Ck;
+    a.out_perm = cluster->out_perm;
+  }
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, s->d, s->L, a.g.BH, 128) || !make_map(&mk, k, s->d, s->L, a.g.BH, 64) ||
       !make_map(&mv, v, s->d, s->L, a.g.BH, 64))
@@ -580,6 +593,153 @@ svg_status svg_attention_step(const svg_shape* s, const svg_params* p, const uin
   if ((st = svg_block_sparse_attn(s, p, qp, kp, vp, kinds, row_ptr, col, full, op, nullptr, stream)) != SVG_OK)
     return st;
   return svg_inverse_layout(s, kinds, op, out, stream);
+}
+
+// ------------------------------------------- semantic-aware permutation (SVG2)
+
+size_t svg2_kmeans_workspace_size(const svg_shape* s, int C) {
+  if (!s || C < 1) return 0;
+  return static_cast<size_t>(s->B) * s->H * C * s->d * sizeof(unsigned long long);
+}
+
+svg_status svg2_kmeans(const svg_shape* s, const uint16_t* x, int C, int iters, int init, float* cent,
+                       uint8_t* assign, int32_t* counts, void* workspace, size_t workspace_bytes, void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  const int Lv = s->F * s->Hs * s->Ws;
+  if (!x || !cent || !assign || !counts || !workspace) return SVG_ERR_INVALID_ARG;
+  if (C < 1 || C > kMaxClusters || C > Lv || iters < 0) return SVG_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, cent, workspace};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return SVG_ERR_ALIGNMENT;
+  if (workspace_bytes < svg2_kmeans_workspace_size(s, C)) return SVG_ERR_CAPACITY;
+  KmArgs a{};
+  a.BH = s->B * s->H;
+  a.L = s->L;
+  a.Lv = Lv;
+  a.C = C;
+  a.x = x;
+  a.cent = cent;
+  a.assign = assign;
+  a.counts = counts;
+  a.sum = static_cast<unsigned long long*>(workspace);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * a.BH * C, cs) != cudaSuccess) return SVG_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, svg2_kmeans_workspace_size(s, C), cs) != cudaSuccess) return SVG_ERR_CUDA;
+  const dim3 cgrid(C, a.BH), agrid((Lv + 255) / 256, a.BH), sgrid((Lv + kKmUpdateRows - 1) / kKmUpdateRows, a.BH);
+  const int asmem = C * s->d * 4, ssmem = C * s->d * 8;
+  auto run = [&](auto D_) -> svg_status {
+    constexpr int D = decltype(D_)::value;
+    if (!set_smem(km_assign_kernel<D>, asmem) || !set_smem(km_sum_kernel<D>, ssmem)) return SVG_ERR_CUDA;
+    if (init) km_init_kernel<D><<<cgrid, D, 0, cs>>>(a);
+    for (int t = 0; t < iters; t++) {
+      km_assign_kernel<D><<<agrid, 256, asmem, cs>>>(a);
+      km_sum_kernel<D><<<sgrid, 256, ssmem, cs>>>(a);
+      km_mean_kernel<D><<<cgrid, D, 0, cs>>>(a);
+    }
+    km_assign_kernel<D><<<agrid, 256, asmem, cs>>>(a);
+    return launch_status();
+  };
+  return s->d == 128 ? run(std::integral_constant<int, 128>{}) : run(std::integral_constant<int, 64>{});
+}
+
+svg_status svg2_permutation(const svg_shape* s, const uint8_t* assign, int C, int32_t* perm, int32_t* off,
+                            void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if (!assign || !perm || !off || C < 1 || C > kMaxClusters) return SVG_ERR_INVALID_ARG;
+  const int Lv = s->F * s->Hs * s->Ws;
+  km_perm_kernel<<<s->B * s->H, 1024, 0, static_cast<cudaStream_t>(stream)>>>(assign, Lv, C, perm, off);
+  return launch_status();
+}
+
+svg_status svg2_select(const svg_shape* s, const svg_params* p, const float* cq, const float* ck,
+                       const int32_t* counts_k, int Cq, int Ck, double top_p, uint64_t* sel, void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if ((st = check_params(s, p, false)) != SVG_OK) return st;
+  if (!cq || !ck || !counts_k || !sel) return SVG_ERR_INVALID_ARG;
+  if (Cq < 1 || Cq > kMaxClusters || Ck < 1 || Ck > kMaxClusters) return SVG_ERR_INVALID_ARG;
+  if (!(top_p > 0.0) || !(top_p <= 1.0)) return SVG_ERR_INVALID_ARG;
+  const double scale = p->softmax_scale > 0.f ? static_cast<double>(p->softmax_scale) : 1.0 / std::sqrt(static_cast<double>(s->d));
+  km_select_kernel<<<dim3(Cq, s->B * s->H), 64, 0, static_cast<cudaStream_t>(stream)>>>(cq, ck, counts_k, Cq, Ck,
+                                                                                        s->d, scale, top_p, sel);
+  return launch_status();
+}
+
+svg_status svg2_permute(const svg_shape* s, const int32_t* perm_q, const int32_t* perm_k, const uint16_t* q,
+                        const uint16_t* k, const uint16_t* v, uint16_t* q_out, uint16_t* k_out, uint16_t* v_out,
+                        void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if (!perm_q || !perm_k || !q || !k || !v || !q_out || !k_out || !v_out) return SVG_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, q_out, k_out, v_out};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return SVG_ERR_ALIGNMENT;
+  if (q == q_out || k == k_out || v == v_out) return SVG_ERR_INVALID_ARG;
+  RowmapArgs a{};
+  a.g = make_geometry(s, nullptr);
+  a.flags = SVG_LAYOUT;
+  a.ntensor = 3;
+  a.norm_tensors = 0;
+  const uint16_t* src[3] = {q, k, v};
+  uint16_t* dst[3] = {q_out, k_out, v_out};
+  const int32_t* gi[3] = {perm_q, perm_k, perm_k};
+  for (int t = 0; t < 3; t++) {
+    a.src[t] = src[t];
+    a.dst[t] = dst[t];
+    a.gather[t] = gi[t];
+  }
+  a.rope = make_rope_args(s, nullptr, nullptr);
+  return launch_rowmap(a, s->d, static_cast<cudaStream_t>(stream));
+}
+
+svg_status svg2_build_block_index(const svg_shape* s, const svg_params* p, int Cq, int Ck, const int32_t* qoff,
+                                  const int32_t* koff, const uint64_t* sel, int32_t* row_ptr, int32_t* col,
+                                  uint8_t* full, int64_t capacity, void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if ((st = check_params(s, p, true)) != SVG_OK) return st;
+  if (!qoff || !koff || !sel || !row_ptr || !col || !full || capacity < 0) return SVG_ERR_INVALID_ARG;
+  if (Cq < 1 || Cq > kMaxClusters || Ck < 1 || Ck > kMaxClusters) return SVG_ERR_INVALID_ARG;
+  const Geometry g0 = make_geometry(s, p);
+  Km2Geom g{};
+  g.BH = g0.BH;
+  g.L = g0.L;
+  g.Lv = g0.Lv;
+  g.bq = g0.bq;
+  g.bk = g0.bk;
+  g.nqb = g0.nqb;
+  g.nkb = g0.nkb;
+  g.Cq = Cq;
+  g.Ck = Ck;
+  g.qoff = qoff;
+  g.koff = koff;
+  g.sel = sel;
+  const int64_t n = static_cast<int64_t>(g.BH) * g.nqb;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  km2_count_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, cs>>>(g, row_ptr);
+  if ((st = launch_status()) != SVG_OK) return st;
+  block_scan_kernel<<<1, 1024, 0, cs>>>(row_ptr, n, capacity);
+  if ((st = launch_status()) != SVG_OK) return st;
+  km2_fill_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, cs>>>(g, row_ptr, col, full, capacity);
+  return launch_status();
+}
+
+svg_status svg2_attention(const svg_shape* s, const svg_params* p, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, int Cq, int Ck, const int32_t* qoff, const int32_t* koff,
+                          const uint64_t* sel, const int32_t* perm_q, const int32_t* row_ptr, const int32_t* col,
+                          const uint8_t* full, uint16_t* out, float* lse_out, void* stream) {
+  if (!qoff || !koff || !sel) return SVG_ERR_INVALID_ARG;
+  if (Cq < 1 || Cq > kMaxClusters || Ck < 1 || Ck > kMaxClusters) return SVG_ERR_INVALID_ARG;
+  AttnArgs c{};
+  c.sel = sel;
+  c.qoff = qoff;
+  c.koff = koff;
+  c.Cq = Cq;
+  c.Ck = Ck;
+  c.out_perm = perm_q;
+  return attention_launch(s, p, q, k, v, nullptr, row_ptr, col, full, out, lse_out, 0, stream, &c);
 }
 
 }  // extern "C"

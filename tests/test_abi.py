@@ -23,7 +23,7 @@ def L():
 def declared_symbols():
     src = open(os.path.join(ROOT, "include", "svg.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(svg_[a-z0-9_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(svg2?_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_every_declared_symbol_is_exported(L):
