@@ -406,7 +406,7 @@ def run_svg2(args):
         mark(5)
         out = svg.svg2_attention(pb, qp, kp, vp, qoff, koff, sel, pq, rp, col, full)
         mark(6)
-        st.update(rp=rp, col=col, sel=sel, out=out)
+        st.update(rp=rp, col=col, sel=sel, out=out, nq=nq, nk=nk)
 
     names = ("qk_norm_rope", "kmeans_q_k", "sort_select", "permute", "block_index", "attention")
     for _ in range(args.warmup):
@@ -414,7 +414,13 @@ def run_svg2(args):
     svg.sync_status()
     n_ent = int(st["rp"][-1])
     flops = kept_tile_flops(st["rp"].cpu().numpy(), st["col"][:n_ent].cpu().numpy(), wl)
-    sel_bits = np.array([bin(int(x)).count("1") for x in st["sel"].cpu().numpy().view(np.uint64).ravel()])
+    sel_np = st["sel"].cpu().numpy().view(np.uint64)
+    sel_bits = np.array([bin(int(x)).count("1") for x in sel_np.ravel()])
+    # kept (query, key) pairs from the cluster sizes: a video query of cluster i keeps
+    # the keys of its selected clusters and the text keys; a text query keeps all
+    nq_np, nk_np = st["nq"].cpu().numpy().astype(np.int64), st["nk"].cpu().numpy().astype(np.int64)
+    bits = ((sel_np[:, :, None] >> np.arange(Ck, dtype=np.uint64)) & np.uint64(1)).astype(np.int64)
+    kept_pairs = float(((nq_np * ((bits * nk_np[:, None, :]).sum(-1) + wl.T)).sum()) + wl.B * wl.H * wl.T * wl.L)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     torch.cuda.synchronize()
     with ClockSampler(0) as clk:
@@ -430,7 +436,7 @@ def run_svg2(args):
     pk, pk_src = peaks()
     attn_tflops = flops / (stage_ms["attention"] * 1e-3) / 1e12
     BH, Lv, d = wl.B * wl.H, wl.Lv, wl.d
-    # one assignment pass: Lv*C*d (subtract, multiply-add) pairs per head and tensor
+    # element-pairs of the assignments: (iters + 1) passes of Lv*C*d per head, for Q and for K
     assign_pairs = 2.0 * BH * Lv * Cq * d * (iters + 1)
     line = {
         "metric": "SVG2 layer ms and effective TFLOP/s over kept tiles",
@@ -441,9 +447,16 @@ def run_svg2(args):
                    "clusters_q": Cq, "clusters_k": Ck, "kmeans_iters": iters, "top_p": top_p,
                    "kept_tile_tflop": round(flops / 1e12, 4),
                    "tile_density": round(n_ent / (BH * wl.nqb * wl.nkb), 4),
+                   "token_density": round(kept_pairs / (BH * float(wl.L) ** 2), 4),
                    "mean_key_clusters_selected": round(float(sel_bits.mean()), 2)},
         "stage_ms": {n: round(t, 4) for n, t in stage_ms.items()},
-        "kmeans_pair_rate_g_per_s": round(assign_pairs / (stage_ms["kmeans_q_k"] * 1e-3) / 1e9, 1),
+        # fp32 ALU bound of the assignment: one subtraction and one FMA per (row, centroid,
+        # dimension); 148 SMs x 128 fp32 lanes x 1965 MHz = 37.2 T lane-ops/s
+        "kmeans_roofline": {"bound": "alu", "unit": "G element-pairs/s",
+                            "achieved": round(assign_pairs / (stage_ms["kmeans_q_k"] * 1e-3) / 1e9, 1),
+                            "peak": round(148 * 128 * 1.965e9 / 2 / 1e9, 1),
+                            "frac": round(assign_pairs / (stage_ms["kmeans_q_k"] * 1e-3) / (148 * 128 * 1.965e9 / 2), 4),
+                            "note": "whole k-means stage (assign, sums, means) over the assignment work alone"},
         "roofline": {"kernel": f"attn2_kernel<{d}> (svg2_attention)", "bound": "tensor",
                      "achieved": round(attn_tflops, 2), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                      "frac": round(attn_tflops / pk["bf16_tflops_sustained"], 4),

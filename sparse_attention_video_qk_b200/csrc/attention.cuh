@@ -81,10 +81,11 @@ struct AttnArgs {
 // layout): the row itself, or, with model_order, its frame-major position --
 // the inverse layout transform (temporal heads: s*F+f -> f*S+s; text rows
 // stay) -- or, with out_perm, the video row the cluster sort put there.
+template <bool CLUSTER>
 __device__ __forceinline__ int out_row(const AttnArgs& a, int kind, int bh, int row) {
   const Geometry& g = a.g;
   if (row >= g.Lv) return row;
-  if (a.out_perm) return a.out_perm[static_cast<int64_t>(bh) * g.Lv + row];
+  if constexpr (CLUSTER) return a.out_perm[static_cast<int64_t>(bh) * g.Lv + row];
   if (!a.model_order || kind != SVG_HEAD_TEMPORAL) return row;
   const int s = row / g.F, f = row - s * g.F;
   return f * g.S + s;
@@ -426,7 +427,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     if (ok && nT > 0 && __all_sync(0xffffffffu, mbar_wait(b_o, (nT - 1) & 1, abort_flag))) {
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row(a, kind, bh, row);
+      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row<false>(a, kind, bh, row);
       uint16_t* orow = a.out + orow_i * D;
 #pragma unroll
       for (int c = 0; c < D / 32; c++) {
@@ -448,7 +449,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       }
       if (row_ok && a.lse) a.lse[orow_i] = (l > 0.f) ? (m_use * 0.69314718055994531f + logf(l)) : -INFINITY;
     } else if (ok && nT == 0 && row_ok) {
-      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row(a, kind, bh, row);
+      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row<false>(a, kind, bh, row);
       uint4* dst = reinterpret_cast<uint4*>(a.out + orow_i * D);
       for (int v = 0; v < D / 8; v++) dst[v] = make_uint4(0, 0, 0, 0);
       if (a.lse) a.lse[orow_i] = -INFINITY;

@@ -78,7 +78,10 @@ struct UnionCursor {
   }
 };
 
-template <int D>
+// CLUSTER: the semantic-permutation mask (a.sel, a.qoff, a.koff, a.out_perm)
+// instead of the head kinds' windows; a separate instantiation, so the window
+// path carries none of its code.
+template <int D, bool CLUSTER>
 __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
     attn2_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                  const __grid_constant__ CUtensorMap tmv, const AttnArgs a) {
@@ -271,13 +274,13 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
     const int q4 = warp & 3;                       // TMEM lane quarter
     const int r = q4 * 32 + lane;
     const int row = (qb0 + w) * g.bq + r;
-    const int kind = a.sel ? static_cast<int>(SVG_HEAD_DENSE) : a.kind[bh];
+    const int kind = CLUSTER ? static_cast<int>(SVG_HEAD_DENSE) : a.kind[bh];
     int lo, hi;
     row_interval(g, kind, row, lo, hi);
     // semantic-permutation mask: this row's key-cluster set (text rows: all)
     uint64_t rmask = ~0ull;
     const int32_t* ko = nullptr;
-    if (a.sel) {
+    if constexpr (CLUSTER) {
       ko = a.koff + static_cast<int64_t>(bh) * (a.Ck + 1);
       if (row < g.Lv)
         rmask = a.sel[static_cast<int64_t>(bh) * a.Cq + cluster_of(a.qoff + static_cast<int64_t>(bh) * (a.Cq + 1),
@@ -326,21 +329,26 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
           for (int c = 0; c < 32; c++) v[c] = __float_as_uint(-INFINITY);
         } else if (mode[h] == 1) {
           const int k0 = kbs[h] * 64 + (q & 1) * 32;
-          if (ko) {
-            // key clusters are contiguous: walk their boundaries along the 32 columns
-            int jc = (k0 < g.Lv) ? cluster_of(ko, a.Ck, k0) : 0;
-            int next = ko[jc + 1];
-            for (int c = 0; c < 32; c++) {
-              const int kk = k0 + c;
-              bool keep;
-              if (kk >= g.Lv) {
-                keep = kk < g.L;
-              } else {
-                while (kk >= next) next = ko[++jc + 1];
-                keep = (rmask >> jc) & 1ull;
+          if constexpr (CLUSTER) {
+            // Key clusters are contiguous, so the 32 columns are a few runs of one
+            // cluster each; the runs are the same for the whole warp.  A run is
+            // kept iff its cluster is in this row's set; text columns always,
+            // columns past L never.
+            uint32_t keep = 0;
+            const int vend = min(k0 + 32, g.Lv);
+            if (k0 < vend) {
+              int jc = cluster_of(ko, a.Ck, k0);          // ko[jc] <= s0 < ko[Ck] = Lv
+              for (int s0 = k0; s0 < vend; jc++) {
+                const int e = min(__ldg(ko + jc + 1), vend);
+                if ((rmask >> jc) & 1ull) keep |= span_bits(s0 - k0, e - k0);
+                s0 = e;
               }
-              if (!keep) v[c] = __float_as_uint(-INFINITY);
             }
+            const int t0 = max(k0, g.Lv), t1 = min(k0 + 32, g.L);
+            if (t0 < t1) keep |= span_bits(t0 - k0, t1 - k0);
+#pragma unroll
+            for (int c = 0; c < 32; c++)
+              if (!((keep >> c) & 1u)) v[c] = __float_as_uint(-INFINITY);
           } else {
 #pragma unroll
             for (int c = 0; c < 32; c++) {
@@ -466,7 +474,7 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
     if (ok && nT > 0 && __all_sync(0xffffffffu, mbar_wait(b_o(w), (nT - 1) & 1, abort_flag))) {
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row(a, kind, bh, row);
+      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row<CLUSTER>(a, kind, bh, row);
       uint16_t* orow = a.out + orow_i * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; c++) {
@@ -488,7 +496,7 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
       }
       if (row_ok && a.lse) a.lse[orow_i] = (l > 0.f) ? (m_use * 0.69314718055994531f + logf(l)) : -INFINITY;
     } else if (ok && nT == 0 && row_ok) {
-      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row(a, kind, bh, row);
+      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row<CLUSTER>(a, kind, bh, row);
       uint4* dst = reinterpret_cast<uint4*>(a.out + orow_i * D);
       for (int v = 0; v < D / 8; v++) dst[v] = make_uint4(0, 0, 0, 0);
       if (a.lse) a.lse[orow_i] = -INFINITY;

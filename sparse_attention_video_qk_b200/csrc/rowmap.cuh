@@ -39,7 +39,6 @@ struct RowmapArgs {
   uint16_t* dst[3];
   const float* gamma[3];     // gains of the normalised tensors
   const uint8_t* kind;       // [B*H], needed when rows move
-  const int32_t* gather[3];  // per tensor or null: destination video row p takes source row gather[bh*Lv + p]
   int rope_floats;           // table size in floats
   RopeArgs rope;             // table in global memory
   FastDiv divF;
@@ -79,8 +78,7 @@ __global__ void __launch_bounds__(256, kRowmapBlocksPerSM) rowmap_kernel(const R
     const int th = unit / nchunk, ch = unit - th * nchunk;
     const int t = th / g.BH, bh = th - t * g.BH;
     const bool norm = t < a.norm_tensors;
-    const int32_t* gidx = a.gather[t] ? a.gather[t] + static_cast<int64_t>(bh) * g.Lv : nullptr;
-    const bool temporal = !gidx && moves && a.kind[bh] == SVG_HEAD_TEMPORAL;
+    const bool temporal = moves && a.kind[bh] == SVG_HEAD_TEMPORAL;
     uint64_t gam[4] = {0ull, 0ull, 0ull, 0ull};
     if (norm) load_gain(a.gamma[t], c, gam);
     const int64_t hbase = static_cast<int64_t>(bh) * g.L;
@@ -96,9 +94,7 @@ __global__ void __launch_bounds__(256, kRowmapBlocksPerSM) rowmap_kernel(const R
         const int p = base + u * RPW + sub;   // destination row in this head
         valid[u] = p < row_end;
         int src_p = p;
-        if (gidx && p < g.Lv) {
-          src_p = valid[u] ? __ldg(gidx + p) : 0;   // semantic permutation (clusters contiguous)
-        } else if (temporal && p < g.Lv) {
+        if (temporal && p < g.Lv) {
           if (inverse) {                      // destination frame-major f*S+s <- s*F+f
             const int f = fdiv(p, a.rope.divS), s = p - f * g.S;
             src_p = s * g.F + f;

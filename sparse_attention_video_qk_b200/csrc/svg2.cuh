@@ -46,14 +46,31 @@ __global__ void km_init_kernel(const KmArgs a) {
 }
 
 // Nearest centroid of every video row, and the cluster sizes.  One thread per
-// row; the head's centroids sit in shared memory (C*D floats).
+// row, the row held in registers as packed bf16 pairs.  The head's centroids
+// sit in shared memory as interleaved pairs, cp[pair][i] = (c_{2 pair}[i],
+// c_{2 pair + 1}[i]), so one 16-byte broadcast load gives two dimensions of
+// two centroids; a pass covers kKmGroup pairs (8 centroids) with one
+// unpacking of each x_i.  Per centroid the distance is still summed over
+// i = 0..D-1 in order, and centroids are compared in index order.
+constexpr int kKmGroup = 4;                              // centroid pairs per pass
+
+__host__ __device__ constexpr int km_assign_pairs(int C) {
+  return (C + 2 * kKmGroup - 1) / (2 * kKmGroup) * kKmGroup;   // padded to whole passes
+}
+
 template <int D>
-__global__ void __launch_bounds__(256) km_assign_kernel(const KmArgs a) {
-  extern __shared__ float cs[];                       // [C][D]
+__global__ void __launch_bounds__(256, D == 128 ? 1 : 2) km_assign_kernel(const KmArgs a) {
+  extern __shared__ float4 cp4[];                     // [pairs][D/2] of (c0[i], c1[i], c0[i+1], c1[i+1])
   __shared__ int cnt[kMaxClusters];
+  float* cpf = reinterpret_cast<float*>(cp4);
   const int bh = blockIdx.y;
-  const int C = a.C;
-  for (int i = threadIdx.x; i < C * D; i += blockDim.x) cs[i] = a.cent[static_cast<int64_t>(bh) * C * D + i];
+  const int C = a.C, npair = km_assign_pairs(C);
+  const float* cg = a.cent + static_cast<int64_t>(bh) * C * D;
+  for (int e = threadIdx.x; e < npair * D * 2; e += blockDim.x) {
+    const int pr = e / (2 * D), rem = e - pr * 2 * D, i = rem >> 1, side = rem & 1;
+    const int c = min(2 * pr + side, C - 1);           // padding repeats the last centroid
+    cpf[e] = cg[c * D + i];
+  }
   if (threadIdx.x < kMaxClusters) cnt[threadIdx.x] = 0;
   __syncthreads();
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
@@ -70,27 +87,38 @@ __global__ void __launch_bounds__(256) km_assign_kernel(const KmArgs a) {
     }
     int best = 0;
     float bestd = INFINITY;
-    for (int c = 0; c < C; c += 2) {
-      // two centroids at once: lanes (c, c+1) of packed pairs, same order as one at a time
-      const float* c0 = cs + c * D;
-      const float* c1 = cs + min(c + 1, C - 1) * D;
-      uint64_t acc = pack_f2(0.f, 0.f);
+    for (int g = 0; g < npair; g += kKmGroup) {
+      uint64_t acc[kKmGroup];
 #pragma unroll
-      for (int i = 0; i < D; i++) {
-        const float xi = (i & 1) ? bf16_hi(xw[i >> 1]) : bf16_lo(xw[i >> 1]);
-        uint64_t t;
-        asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(pack_f2(xi, xi)), "l"(pack_f2(c0[i], c1[i])));
-        acc = fma_f2(t, t, acc);
+      for (int p = 0; p < kKmGroup; p++) acc[p] = pack_f2(0.f, 0.f);
+      const float4* base = cp4 + g * (D / 2);
+#pragma unroll
+      for (int j = 0; j < D / 2; j++) {                 // dimensions 2j, 2j+1
+        const float xa = bf16_lo(xw[j]), xb = bf16_hi(xw[j]);
+        const uint64_t xa2 = pack_f2(xa, xa), xb2 = pack_f2(xb, xb);
+#pragma unroll
+        for (int p = 0; p < kKmGroup; p++) {
+          const float4 c = base[p * (D / 2) + j];
+          uint64_t t;
+          asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(xa2), "l"(pack_f2(c.x, c.y)));
+          acc[p] = fma_f2(t, t, acc[p]);
+          asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(xb2), "l"(pack_f2(c.z, c.w)));
+          acc[p] = fma_f2(t, t, acc[p]);
+        }
       }
-      float d0, d1;
-      unpack_f2(acc, d0, d1);
-      if (d0 < bestd) {
-        bestd = d0;
-        best = c;
-      }
-      if (c + 1 < C && d1 < bestd) {
-        bestd = d1;
-        best = c + 1;
+#pragma unroll
+      for (int p = 0; p < kKmGroup; p++) {
+        const int c = 2 * (g + p);
+        float d0, d1;
+        unpack_f2(acc[p], d0, d1);
+        if (c < C && d0 < bestd) {
+          bestd = d0;
+          best = c;
+        }
+        if (c + 1 < C && d1 < bestd) {
+          bestd = d1;
+          best = c + 1;
+        }
       }
     }
     a.assign[static_cast<int64_t>(bh) * a.Lv + r] = static_cast<uint8_t>(best);
@@ -239,6 +267,55 @@ __global__ void __launch_bounds__(64) km_select_kernel(const float* __restrict__
   }
 }
 
+// ------------------------------------------------------- permutation of Q, K, V
+
+struct KmGatherArgs {
+  int BH, L, Lv;
+  FastDiv divL;
+  const uint16_t* src[3];
+  uint16_t* dst[3];
+  const int32_t* perm[3];  // [BH][Lv]: video position p of dst takes row perm[p] of src
+};
+
+// dst row p <- src row perm[p] (video rows), text rows copied in place.
+// One 16-byte chunk per thread and step, kKmGatherU steps in flight; the
+// stores are coalesced, a source row is read whole (D*2 contiguous bytes).
+// blockIdx.y = tensor.
+constexpr int kKmGatherU = 4;
+
+template <int D>
+__global__ void __launch_bounds__(256) km_gather_kernel(const KmGatherArgs a) {
+  constexpr int CH = D / 8;                           // 16-byte chunks per row
+  constexpr int SH = (D == 128) ? 4 : 3;
+  static_assert((1 << SH) == CH, "chunks per row");
+  // select the tensor without indexing the parameter arrays dynamically (that
+  // would copy them to local memory)
+  const int t = blockIdx.y;
+  const uint4* __restrict__ src = reinterpret_cast<const uint4*>(t == 0 ? a.src[0] : t == 1 ? a.src[1] : a.src[2]);
+  uint4* __restrict__ dst = reinterpret_cast<uint4*>(t == 0 ? a.dst[0] : t == 1 ? a.dst[1] : a.dst[2]);
+  const int32_t* __restrict__ perm = t == 0 ? a.perm[0] : t == 1 ? a.perm[1] : a.perm[2];
+  const int64_t n = static_cast<int64_t>(a.BH) * a.L * CH;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < n; i0 += step * kKmGatherU) {
+    uint4 x[kKmGatherU];
+#pragma unroll
+    for (int u = 0; u < kKmGatherU; u++) {
+      const int64_t i = i0 + u * step;
+      if (i < n) {
+        const int row = static_cast<int>(i >> SH), c = static_cast<int>(i & (CH - 1));
+        const int bh = fdiv(row, a.divL), p = row - bh * a.L;
+        const int sp = (p < a.Lv) ? __ldg(perm + static_cast<int64_t>(bh) * a.Lv + p) : p;
+        x[u] = __ldg(src + (static_cast<int64_t>(bh) * a.L + sp) * CH + c);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kKmGatherU; u++) {
+      const int64_t i = i0 + u * step;
+      if (i < n) dst[i] = x[u];
+    }
+  }
+}
+
 // ------------------------------------------------ block index, permuted order
 
 struct Km2Geom {
@@ -248,66 +325,83 @@ struct Km2Geom {
   const uint64_t* sel;     // [BH][Cq]
 };
 
-// Walks the key blocks of one query tile and calls f(kb, full) for every
-// listed one.  In the permuted order a query tile covers a run of query
-// clusters and a key block a run of key clusters; a pair (i, j) is kept iff bit
-// j of sel[i] is set, text keys are kept by every query, text queries keep
-// every key.  U / I = OR / AND of sel over the tile's query clusters.
-template <typename Fn>
-__device__ __forceinline__ void km2_tile_walk(const Km2Geom& g, int bh, int qb, Fn f) {
+// One warp per (head, query tile).  In the permuted order a query tile covers a
+// run of query clusters and a key block a run of key clusters; a pair (i, j)
+// is kept iff bit j of sel[i] is set, text keys are kept by every query and
+// text queries keep every key.  With U / I = OR / AND of sel over the tile's
+// non-empty query clusters and R = the key clusters present in a block, the
+// block is listed iff it holds a text key or U & R != 0, and full iff every
+// pair is kept: the tile has no video query or I covers R.  The lanes take
+// the key blocks 32 apart; ballots give the count and each entry's slot, so
+// the list comes out in increasing block order.
+struct Km2Tile {
+  uint64_t U, I;
+  bool video_q;
+};
+
+__device__ __forceinline__ Km2Tile km2_tile(const Km2Geom& g, int bh, int qb) {
   const int32_t* qo = g.qoff + static_cast<int64_t>(bh) * (g.Cq + 1);
-  const int32_t* ko = g.koff + static_cast<int64_t>(bh) * (g.Ck + 1);
   const uint64_t* sl = g.sel + static_cast<int64_t>(bh) * g.Cq;
   const int q0 = qb * g.bq, q1 = min(g.L, q0 + g.bq);
-  const bool text_q = q1 > g.Lv, video_q = q0 < g.Lv;
-  uint64_t U = 0, I = ~0ull;
-  if (video_q) {
+  Km2Tile t{0ull, ~0ull, q0 < g.Lv};
+  if (t.video_q) {
     const int i0 = cluster_of(qo, g.Cq, q0), i1 = cluster_of(qo, g.Cq, min(q1, g.Lv) - 1);
     for (int i = i0; i <= i1; i++)
-      if (qo[i + 1] > qo[i]) {
-        U |= sl[i];
-        I &= sl[i];
+      if (__ldg(qo + i + 1) > __ldg(qo + i)) {
+        const uint64_t m = __ldg(reinterpret_cast<const unsigned long long*>(sl) + i);
+        t.U |= m;
+        t.I &= m;
       }
   }
-  if (text_q) U = ~0ull;
-  int j = 0;                                   // key cluster of the current block's first video key
-  for (int kb = 0; kb < g.nkb; kb++) {
-    const int k0 = kb * g.bk, k1 = min(g.L, k0 + g.bk);
-    const bool text_k = k1 > g.Lv;
-    uint64_t R = 0;                            // non-empty key clusters in the block
-    if (k0 < g.Lv) {
-      while (ko[j + 1] <= k0) j++;
-      for (int t = j; t < g.Ck && ko[t] < min(k1, g.Lv); t++)
-        if (ko[t + 1] > ko[t]) R |= 1ull << t;
+  if (q1 > g.Lv) t.U = ~0ull;                   // a text query keeps every key
+  return t;
+}
+
+// Key clusters present in video keys [k0, k1) of one head (0 if none).
+__device__ __forceinline__ uint64_t km2_block_clusters(const Km2Geom& g, const int32_t* ko, int k0, int k1) {
+  uint64_t R = 0;
+  const int e = min(k1, g.Lv);
+  if (k0 < e)
+    for (int j = cluster_of(ko, g.Ck, k0); j < g.Ck && __ldg(ko + j) < e; j++)
+      if (__ldg(ko + j + 1) > __ldg(ko + j)) R |= 1ull << j;
+  return R;
+}
+
+template <bool FILL>
+__global__ void __launch_bounds__(256, 4) km2_list_kernel(const Km2Geom g, int32_t* __restrict__ row_ptr,
+                                                       int32_t* __restrict__ col, uint8_t* __restrict__ full,
+                                                       int64_t capacity) {
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t n = static_cast<int64_t>(g.BH) * g.nqb;
+  if (wid >= n) return;                          // whole warps leave together
+  const int bh = static_cast<int>(wid / g.nqb), qb = static_cast<int>(wid % g.nqb);
+  const Km2Tile t = km2_tile(g, bh, qb);
+  const int32_t* ko = g.koff + static_cast<int64_t>(bh) * (g.Ck + 1);
+  int64_t e = FILL ? static_cast<int64_t>(row_ptr[wid]) : 0;
+  for (int kb0 = 0; kb0 < g.nkb; kb0 += 32) {
+    const int kb = kb0 + lane;
+    bool listed = false, fl = false;
+    if (kb < g.nkb) {
+      const int k0 = kb * g.bk, k1 = min(g.L, k0 + g.bk);
+      const uint64_t R = km2_block_clusters(g, ko, k0, k1);
+      listed = (k1 > g.Lv) || (t.U & R) != 0;
+      fl = !t.video_q || (t.I & R) == R;
     }
-    const bool listed = text_k || (U & R) != 0;
-    if (listed) f(kb, (!video_q || (I & R) == R) ? 1 : 0);
+    const unsigned b = __ballot_sync(0xffffffffu, listed);
+    if (FILL && listed) {
+      const int64_t slot = e + __popc(b & ((1u << lane) - 1u));
+      if (slot < capacity) {
+        col[slot] = kb;
+        full[slot] = fl ? 1 : 0;
+      }
+    }
+    e += __popc(b);
   }
-}
-
-__global__ void km2_count_kernel(const Km2Geom g, int32_t* __restrict__ row_ptr) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t n = static_cast<int64_t>(g.BH) * g.nqb;
-  if (i >= n) return;
-  int cnt = 0;
-  km2_tile_walk(g, static_cast<int>(i / g.nqb), static_cast<int>(i % g.nqb), [&](int, int) { cnt++; });
-  row_ptr[i + 1] = cnt;
-  if (i == 0) row_ptr[0] = 0;
-}
-
-__global__ void km2_fill_kernel(const Km2Geom g, const int32_t* __restrict__ row_ptr, int32_t* __restrict__ col,
-                                uint8_t* __restrict__ full, int64_t capacity) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t n = static_cast<int64_t>(g.BH) * g.nqb;
-  if (i >= n) return;
-  int64_t e = row_ptr[i];
-  km2_tile_walk(g, static_cast<int>(i / g.nqb), static_cast<int>(i % g.nqb), [&](int kb, int fl) {
-    if (e < capacity) {
-      col[e] = kb;
-      full[e] = static_cast<uint8_t>(fl);
-    }
-    e++;
-  });
+  if (!FILL && lane == 0) {
+    row_ptr[wid + 1] = static_cast<int32_t>(e);
+    if (wid == 0) row_ptr[0] = 0;
+  }
 }
 
 }  // namespace svg

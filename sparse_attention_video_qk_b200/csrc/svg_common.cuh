@@ -73,6 +73,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Bits [a, b) of a 32-bit word, 0 <= a < b <= 32.
+__device__ __forceinline__ uint32_t span_bits(int a, int b) {
+  const uint32_t w = (b - a >= 32) ? 0xFFFFFFFFu : ((1u << (b - a)) - 1u);
+  return w << a;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 

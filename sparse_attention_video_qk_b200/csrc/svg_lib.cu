@@ -3,6 +3,7 @@
 // kernels are in the included .cuh files (one translation unit).
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -527,14 +528,19 @@ static svg_status attention_launch(const svg_shape* s, const svg_params* p, cons
   if (a.g.bq == 128) {
     // two 128-row query tiles per CTA share every K/V tile
     const unsigned grid = static_cast<unsigned>(a.g.BH) * static_cast<unsigned>((a.g.nqb + 1) / 2);
+    auto run = [&](auto kern, int threads, int smem) -> svg_status {
+      if (!set_smem(kern, smem)) return SVG_ERR_CUDA;
+      kern<<<grid, threads, smem, cs>>>(mq, mk, mv, a);
+      return launch_status();
+    };
     if (s->d == 128) {
-      if (!set_smem(attn2_kernel<128>, Attn2Cfg<128>::SMEM_BYTES)) return SVG_ERR_CUDA;
-      attn2_kernel<128><<<grid, Attn2Cfg<128>::THREADS, Attn2Cfg<128>::SMEM_BYTES, cs>>>(mq, mk, mv, a);
-    } else {
-      if (!set_smem(attn2_kernel<64>, Attn2Cfg<64>::SMEM_BYTES)) return SVG_ERR_CUDA;
-      attn2_kernel<64><<<grid, Attn2Cfg<64>::THREADS, Attn2Cfg<64>::SMEM_BYTES, cs>>>(mq, mk, mv, a);
+      using C = Attn2Cfg<128>;
+      return cluster ? run(attn2_kernel<128, true>, C::THREADS, C::SMEM_BYTES)
+                     : run(attn2_kernel<128, false>, C::THREADS, C::SMEM_BYTES);
     }
-    return launch_status();
+    using C = Attn2Cfg<64>;
+    return cluster ? run(attn2_kernel<64, true>, C::THREADS, C::SMEM_BYTES)
+                   : run(attn2_kernel<64, false>, C::THREADS, C::SMEM_BYTES);
   }
   const unsigned grid = static_cast<unsigned>(a.g.BH) * static_cast<unsigned>(a.g.nqb);
   if (s->d == 128) {
@@ -627,7 +633,7 @@ svg_status svg2_kmeans(const svg_shape* s, const uint16_t* x, int C, int iters, 
   if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * a.BH * C, cs) != cudaSuccess) return SVG_ERR_CUDA;
   if (cudaMemsetAsync(workspace, 0, svg2_kmeans_workspace_size(s, C), cs) != cudaSuccess) return SVG_ERR_CUDA;
   const dim3 cgrid(C, a.BH), agrid((Lv + 255) / 256, a.BH), sgrid((Lv + kKmUpdateRows - 1) / kKmUpdateRows, a.BH);
-  const int asmem = C * s->d * 4, ssmem = C * s->d * 8;
+  const int asmem = km_assign_pairs(C) * 2 * s->d * 4, ssmem = C * s->d * 8;
   auto run = [&](auto D_) -> svg_status {
     constexpr int D = decltype(D_)::value;
     if (!set_smem(km_assign_kernel<D>, asmem) || !set_smem(km_sum_kernel<D>, ssmem)) return SVG_ERR_CUDA;
@@ -677,21 +683,27 @@ svg_status svg2_permute(const svg_shape* s, const int32_t* perm_q, const int32_t
   for (const void* ptr : ptrs)
     if (!aligned16(ptr)) return SVG_ERR_ALIGNMENT;
   if (q == q_out || k == k_out || v == v_out) return SVG_ERR_INVALID_ARG;
-  RowmapArgs a{};
-  a.g = make_geometry(s, nullptr);
-  a.flags = SVG_LAYOUT;
-  a.ntensor = 3;
-  a.norm_tensors = 0;
+  KmGatherArgs a{};
+  a.BH = s->B * s->H;
+  a.L = s->L;
+  a.Lv = s->F * s->Hs * s->Ws;
+  a.divL = make_fastdiv(s->L);
   const uint16_t* src[3] = {q, k, v};
   uint16_t* dst[3] = {q_out, k_out, v_out};
-  const int32_t* gi[3] = {perm_q, perm_k, perm_k};
+  const int32_t* pi[3] = {perm_q, perm_k, perm_k};
   for (int t = 0; t < 3; t++) {
     a.src[t] = src[t];
     a.dst[t] = dst[t];
-    a.gather[t] = gi[t];
+    a.perm[t] = pi[t];
   }
-  a.rope = make_rope_args(s, nullptr, nullptr);
-  return launch_rowmap(a, s->d, static_cast<cudaStream_t>(stream));
+  const int64_t units = static_cast<int64_t>(a.BH) * a.L * (s->d / 8);
+  const int64_t per_block = 256LL * kKmGatherU;
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((units + per_block - 1) / per_block, 148LL * 8));
+  const dim3 grid(blocks, 3);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (s->d == 128) km_gather_kernel<128><<<grid, 256, 0, cs>>>(a);
+  else km_gather_kernel<64><<<grid, 256, 0, cs>>>(a);
+  return launch_status();
 }
 
 svg_status svg2_build_block_index(const svg_shape* s, const svg_params* p, int Cq, int Ck, const int32_t* qoff,
@@ -718,11 +730,12 @@ svg_status svg2_build_block_index(const svg_shape* s, const svg_params* p, int C
   g.sel = sel;
   const int64_t n = static_cast<int64_t>(g.BH) * g.nqb;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  km2_count_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, cs>>>(g, row_ptr);
+  const unsigned blocks = static_cast<unsigned>((n * 32 + 255) / 256);   // one warp per query tile
+  km2_list_kernel<false><<<blocks, 256, 0, cs>>>(g, row_ptr, col, full, capacity);
   if ((st = launch_status()) != SVG_OK) return st;
   block_scan_kernel<<<1, 1024, 0, cs>>>(row_ptr, n, capacity);
   if ((st = launch_status()) != SVG_OK) return st;
-  km2_fill_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, cs>>>(g, row_ptr, col, full, capacity);
+  km2_list_kernel<true><<<blocks, 256, 0, cs>>>(g, row_ptr, col, full, capacity);
   return launch_status();
 }
 
