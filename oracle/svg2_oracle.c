@@ -18,9 +18,11 @@
  *   4. attention of each query row to the keys of its selected clusters.
  * The page gives no numbers or precisions.  Readings (also in the design notes):
  *   - init: centroid c = row floor(c * Lv / C); text rows are not clustered;
- *   - a distance is d(x, c) = sum_i (x_i - c_i)^2 accumulated in float in the
- *     order i = 0..d-1 with fused multiply-add; the nearest centroid wins, the
- *     lowest index on a tie.  This decides an integer, so it is taken in the
+ *   - the nearest centroid minimises |c|^2 - 2 x.c (the squared Euclidean
+ *     distance without the |x|^2 term, which is the same for every centroid);
+ *     |c|^2 and x.c are each accumulated in float in the order i = 0..d-1 with
+ *     fused multiply-add, then |c|^2 - 2 (x.c) is rounded once; the lowest
+ *     index wins a tie.  This decides an integer, so it is taken in the
  *     precision the kernel uses;
  *   - a centroid sum is kept in 64-bit fixed point (value * 2^40, truncated
  *     toward zero), so its value does not depend on the order of the rows; the
@@ -75,13 +77,14 @@ void ora2_assign(const uint16_t* x, int BH, int64_t L, int64_t Lv, int d, int C,
     float bestd = INFINITY;
     for (int c = 0; c < C; c++) {
       const float* cc = cent + (bh * C + c) * d;
-      float acc = 0.0f;
+      float cn = 0.0f, dot = 0.0f;
       for (int i = 0; i < d; i++) {
-        float t = bf16_to_f32(xr[i]) - cc[i];
-        acc = fmaf(t, t, acc);
+        cn = fmaf(cc[i], cc[i], cn);
+        dot = fmaf(bf16_to_f32(xr[i]), cc[i], dot);
       }
-      if (acc < bestd) {
-        bestd = acc;
+      const float dist = fmaf(-2.0f, dot, cn);
+      if (dist < bestd) {
+        bestd = dist;
         best = c;
       }
     }
