@@ -450,17 +450,19 @@ def run_svg2(args):
                    "token_density": round(kept_pairs / (BH * float(wl.L) ** 2), 4),
                    "mean_key_clusters_selected": round(float(sel_bits.mean()), 2)},
         "stage_ms": {n: round(t, 4) for n, t in stage_ms.items()},
-        # fp32 ALU bound of the assignment: one subtraction and one FMA per (row, centroid,
-        # dimension); 148 SMs x 128 fp32 lanes x 1965 MHz = 37.2 T lane-ops/s
+        # fp32 ALU bound of the assignment: one FMA per (row, centroid, dimension);
+        # 148 SMs x 128 fp32 lanes x 1965 MHz = 37.2 T FMA/s
         "kmeans_roofline": {"bound": "alu", "unit": "G element-pairs/s",
                             "achieved": round(assign_pairs / (stage_ms["kmeans_q_k"] * 1e-3) / 1e9, 1),
-                            "peak": round(148 * 128 * 1.965e9 / 2 / 1e9, 1),
-                            "frac": round(assign_pairs / (stage_ms["kmeans_q_k"] * 1e-3) / (148 * 128 * 1.965e9 / 2), 4),
+                            "peak": round(148 * 128 * 1.965e9 / 1e9, 1),
+                            "frac": round(assign_pairs / (stage_ms["kmeans_q_k"] * 1e-3) / (148 * 128 * 1.965e9), 4),
                             "note": "whole k-means stage (assign, sums, means) over the assignment work alone"},
         "roofline": {"kernel": f"attn2_kernel<{d}> (svg2_attention)", "bound": "tensor",
                      "achieved": round(attn_tflops, 2), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                      "frac": round(attn_tflops / pk["bf16_tflops_sustained"], 4),
-                     "peak_source": f"{pk_src} bf16 sustained", "traffic": None},
+                     "peak_source": f"{pk_src} bf16 sustained",
+                     "traffic": traffic_from_profile("attention2.cuh", "attention_svg2_hunyuanvideo_720p.md")
+                     if wl == W.HUNYUAN and (Cq, Ck, iters, top_p) == (64, 64, 2, 0.9) else None},
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)

@@ -264,10 +264,12 @@ size_t svg2_kmeans_workspace_size(const svg_shape* shape, int C);
  * `cent` holds the starting centroids (e.g. the previous denoising step's: the
  * pages' centroid cache).  `iters` rounds of (assign every row to its nearest
  * centroid; move each centroid to the mean of its rows, an empty cluster keeps
- * its centroid), then a final assignment.  Distance sum_i (x_i - c_i)^2 in float
- * with fused multiply-add in the order i = 0..d-1, the lowest index on a tie;
- * sums in 64-bit fixed point (x * 2^40 truncated), mean ((double)sum / 2^40) /
- * count rounded to float.
+ * its centroid), then a final assignment.  The nearest centroid minimises
+ * |c|^2 - 2 x.c (the squared distance less |x|^2): both sums in float with
+ * fused multiply-add in the order i = 0..d-1, then |c|^2 - 2 (x.c) rounded
+ * once; the lowest index wins a tie.  Sums in 64-bit fixed point (x * 2^40
+ * truncated), exact while a cluster's sum of |x| stays below 2^23; mean
+ * ((double)sum / 2^40) / count rounded to float.
  * cent: device float [B*H][C][d] (in/out); assign: device uint8 [B*H][Lv];
  * counts: device int32 [B*H][C], the sizes of the final assignment. */
 svg_status svg2_kmeans(const svg_shape* shape, const uint16_t* x, int C, int iters, int init, float* cent,

@@ -7,8 +7,9 @@
 //
 // Decisions made from floating point (nearest centroid, top-p set) are taken
 // with a fixed operation order so that they do not depend on scheduling:
-//   * a distance is sum_i (x_i - c_i)^2 in float, i = 0..d-1, each step one
-//     subtraction and one fused multiply-add (packed over two centroids);
+//   * the nearest centroid minimises |c|^2 - 2 x.c, both sums in float over
+//     i = 0..d-1 with fused multiply-adds (packed over two centroids), then
+//     one rounding of |c|^2 - 2 (x.c);
 //   * centroid sums are 64-bit fixed point (value * 2^40, truncated toward
 //     zero), so atomics in any order give the same sum; the mean is
 //     ((double)sum / 2^40) / count rounded to float; an empty cluster keeps
@@ -45,38 +46,55 @@ __global__ void km_init_kernel(const KmArgs a) {
     a.cent[(static_cast<int64_t>(bh) * a.C + c) * D + i] = __uint_as_float(static_cast<uint32_t>(xr[i]) << 16);
 }
 
-// Nearest centroid of every video row, and the cluster sizes.  One thread per
-// row, the row held in registers as packed bf16 pairs.  The head's centroids
-// sit in shared memory as interleaved pairs, cp[pair][i] = (c_{2 pair}[i],
-// c_{2 pair + 1}[i]), so one 16-byte broadcast load gives two dimensions of
-// two centroids; a pass covers kKmGroup pairs (8 centroids) with one
-// unpacking of each x_i.  Per centroid the distance is still summed over
-// i = 0..D-1 in order, and centroids are compared in index order.
-constexpr int kKmGroup = 4;                              // centroid pairs per pass
+// Nearest centroid of every video row, and the cluster sizes.  The nearest
+// centroid minimises |c|^2 - 2 x.c (the squared distance without |x|^2, the
+// same for every centroid): |c|^2 and x.c are each summed in fp32 over
+// i = 0..D-1 with fused multiply-adds, then |c|^2 - 2 (x.c) is rounded once;
+// centroids are compared in index order, the lowest index winning a tie.
+// Two rows per thread, held in registers as packed bf16 pairs.  The
+// head's centroids sit in shared memory as interleaved pairs,
+// cp[pair][i] = (c_{2 pair}[i], c_{2 pair + 1}[i]), so a 16-byte broadcast
+// load gives two dimensions of two centroids and one packed FMA advances two
+// dot products; a pass covers kKmGroup pairs (8 centroids) with one unpacking
+// of each x_i.
+constexpr int kKmGroup = 4;                              // centroid pairs per pass (padding unit)
 
 __host__ __device__ constexpr int km_assign_pairs(int C) {
   return (C + 2 * kKmGroup - 1) / (2 * kKmGroup) * kKmGroup;   // padded to whole passes
 }
 
+// pairs per pass: fewer at d = 128, where the two rows take 128 registers
 template <int D>
-__global__ void __launch_bounds__(256, D == 128 ? 1 : 2) km_assign_kernel(const KmArgs a) {
-  extern __shared__ float4 cp4[];                     // [pairs][D/2] of (c0[i], c1[i], c0[i+1], c1[i+1])
-  __shared__ int cnt[kMaxClusters];
-  float* cpf = reinterpret_cast<float*>(cp4);
-  const int bh = blockIdx.y;
-  const int C = a.C, npair = km_assign_pairs(C);
-  const float* cg = a.cent + static_cast<int64_t>(bh) * C * D;
-  for (int e = threadIdx.x; e < npair * D * 2; e += blockDim.x) {
-    const int pr = e / (2 * D), rem = e - pr * 2 * D, i = rem >> 1, side = rem & 1;
-    const int c = min(2 * pr + side, C - 1);           // padding repeats the last centroid
-    cpf[e] = cg[c * D + i];
-  }
-  if (threadIdx.x < kMaxClusters) cnt[threadIdx.x] = 0;
-  __syncthreads();
-  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+__host__ __device__ constexpr int km_group() {
+  return D == 128 ? 4 : 4;
+}
+
+// shared memory of km_assign_kernel: the pairs, then |c|^2 of every (padded) centroid
+__host__ __device__ constexpr int km_assign_smem(int C, int D) {
+  return km_assign_pairs(C) * 2 * D * 4 + km_assign_pairs(C) * 2 * 4;
+}
+
+// (lo, lo) and (hi, hi) as packed fp32 pairs from one packed bf16 pair.  The
+// asm is volatile so that the unpacking stays inside the centroid loop:
+// hoisted out of it, the unpacked rows would need 2*D registers per row.
+__device__ __forceinline__ void bf16x2_dup(uint32_t w, uint64_t& lo2, uint64_t& hi2) {
+  asm volatile(
+      "{\n\t.reg .b32 l, h;\n\t"
+      "shl.b32 l, %2, 16;\n\t"
+      "and.b32 h, %2, 0xFFFF0000;\n\t"
+      "mov.b64 %0, {l, l};\n\t"
+      "mov.b64 %1, {h, h};\n\t}"
+      : "=l"(lo2), "=l"(hi2)
+      : "r"(w));
+}
+
+constexpr int kKmAssignThreads = 128;                  // each thread takes two rows
+constexpr int kKmAssignRows = 2 * kKmAssignThreads;     // rows per block
+
+template <int D>
+__device__ __forceinline__ void km_load_row(const KmArgs& a, int bh, int r, uint32_t* xw) {
   if (r < a.Lv) {
     const uint4* xr = reinterpret_cast<const uint4*>(a.x + (static_cast<int64_t>(bh) * a.L + r) * D);
-    uint32_t xw[D / 2];                                 // the row as packed bf16 pairs
 #pragma unroll
     for (int v = 0; v < D / 8; v++) {
       const uint4 u = __ldg(xr + v);
@@ -85,73 +103,172 @@ __global__ void __launch_bounds__(256, D == 128 ? 1 : 2) km_assign_kernel(const 
       xw[4 * v + 2] = u.z;
       xw[4 * v + 3] = u.w;
     }
-    int best = 0;
-    float bestd = INFINITY;
-    for (int g = 0; g < npair; g += kKmGroup) {
-      uint64_t acc[kKmGroup];
+  } else {
 #pragma unroll
-      for (int p = 0; p < kKmGroup; p++) acc[p] = pack_f2(0.f, 0.f);
+    for (int v = 0; v < D / 2; v++) xw[v] = 0u;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kKmAssignThreads, 1) km_assign_kernel(const KmArgs a) {
+  extern __shared__ float4 cp4[];                     // [pairs][D/2] of (c0[i], c1[i], c0[i+1], c1[i+1])
+  __shared__ int cnt[kMaxClusters];
+  float* cpf = reinterpret_cast<float*>(cp4);
+  const int bh = blockIdx.y;
+  const int C = a.C, npair = km_assign_pairs(C);
+  float* cn = cpf + npair * 2 * D;                    // [2 * npair]
+  const float* cg = a.cent + static_cast<int64_t>(bh) * C * D;
+  for (int e = threadIdx.x; e < npair * D * 2; e += blockDim.x) {
+    const int pr = e / (2 * D), rem = e - pr * 2 * D, i = rem >> 1, side = rem & 1;
+    const int c = min(2 * pr + side, C - 1);           // padding repeats the last centroid
+    cpf[e] = cg[c * D + i];
+  }
+  for (int c = threadIdx.x; c < 2 * npair; c += blockDim.x) {
+    const float* cc = cg + min(c, C - 1) * D;
+    float acc = 0.f;
+    for (int i = 0; i < D; i++) acc = fmaf(cc[i], cc[i], acc);
+    cn[c] = acc;
+  }
+  if (threadIdx.x < kMaxClusters) cnt[threadIdx.x] = 0;
+  __syncthreads();
+  // two rows per thread: every centroid value loaded from shared memory feeds both
+  const int r0 = blockIdx.x * kKmAssignRows + threadIdx.x, r1 = r0 + kKmAssignThreads;
+  if (r0 < a.Lv) {
+    uint32_t xw0[D / 2], xw1[D / 2];                    // the rows as packed bf16 pairs
+    km_load_row<D>(a, bh, r0, xw0);
+    km_load_row<D>(a, bh, r1, xw1);
+    int best0 = 0, best1 = 0;
+    float bestd0 = INFINITY, bestd1 = INFINITY;
+    constexpr int G = km_group<D>();
+    for (int g = 0; g < npair; g += G) {
+      uint64_t acc0[G], acc1[G];
+#pragma unroll
+      for (int p = 0; p < G; p++) acc0[p] = acc1[p] = pack_f2(0.f, 0.f);
       const float4* base = cp4 + g * (D / 2);
 #pragma unroll
       for (int j = 0; j < D / 2; j++) {                 // dimensions 2j, 2j+1
-        const float xa = bf16_lo(xw[j]), xb = bf16_hi(xw[j]);
-        const uint64_t xa2 = pack_f2(xa, xa), xb2 = pack_f2(xb, xb);
+        uint64_t xa02, xb02, xa12, xb12;
+        bf16x2_dup(xw0[j], xa02, xb02);
+        bf16x2_dup(xw1[j], xa12, xb12);
 #pragma unroll
-        for (int p = 0; p < kKmGroup; p++) {
+        for (int p = 0; p < G; p++) {
           const float4 c = base[p * (D / 2) + j];
-          uint64_t t;
-          asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(xa2), "l"(pack_f2(c.x, c.y)));
-          acc[p] = fma_f2(t, t, acc[p]);
-          asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(xb2), "l"(pack_f2(c.z, c.w)));
-          acc[p] = fma_f2(t, t, acc[p]);
+          const uint64_t ca = pack_f2(c.x, c.y), cb = pack_f2(c.z, c.w);
+          acc0[p] = fma_f2(xa02, ca, acc0[p]);
+          acc1[p] = fma_f2(xa12, ca, acc1[p]);
+          acc0[p] = fma_f2(xb02, cb, acc0[p]);
+          acc1[p] = fma_f2(xb12, cb, acc1[p]);
         }
       }
 #pragma unroll
-      for (int p = 0; p < kKmGroup; p++) {
+      for (int p = 0; p < G; p++) {
         const int c = 2 * (g + p);
-        float d0, d1;
-        unpack_f2(acc[p], d0, d1);
-        if (c < C && d0 < bestd) {
-          bestd = d0;
-          best = c;
+        float u0, u1, w0, w1;
+        unpack_f2(acc0[p], u0, u1);
+        unpack_f2(acc1[p], w0, w1);
+        const float du0 = fmaf(-2.f, u0, cn[c]), du1 = fmaf(-2.f, u1, cn[c + 1]);
+        const float dw0 = fmaf(-2.f, w0, cn[c]), dw1 = fmaf(-2.f, w1, cn[c + 1]);
+        if (c < C) {
+          if (du0 < bestd0) { bestd0 = du0; best0 = c; }
+          if (dw0 < bestd1) { bestd1 = dw0; best1 = c; }
         }
-        if (c + 1 < C && d1 < bestd) {
-          bestd = d1;
-          best = c + 1;
+        if (c + 1 < C) {
+          if (du1 < bestd0) { bestd0 = du1; best0 = c + 1; }
+          if (dw1 < bestd1) { bestd1 = dw1; best1 = c + 1; }
         }
       }
     }
-    a.assign[static_cast<int64_t>(bh) * a.Lv + r] = static_cast<uint8_t>(best);
-    atomicAdd(&cnt[best], 1);
+    a.assign[static_cast<int64_t>(bh) * a.Lv + r0] = static_cast<uint8_t>(best0);
+    atomicAdd(&cnt[best0], 1);
+    if (r1 < a.Lv) {
+      a.assign[static_cast<int64_t>(bh) * a.Lv + r1] = static_cast<uint8_t>(best1);
+      atomicAdd(&cnt[best1], 1);
+    }
   }
   __syncthreads();
   if (threadIdx.x < C && cnt[threadIdx.x]) atomicAdd(&a.counts[bh * C + threadIdx.x], cnt[threadIdx.x]);
 }
 
 // Fixed-point sums of the rows of every cluster: a block sums a run of rows of
-// one head in shared memory, then adds its sums to the head's global sums.
+// one head in shared memory, then adds its sums to the head's global 64-bit
+// sums.  Each warp walks its own contiguous share of the block's rows (four
+// rows in flight), keeping the running sums of its current cluster in
+// registers and flushing them to shared memory when the cluster changes, so
+// a run of rows in one cluster costs one flush.  A flushed 64-bit value v is
+// split as v = hi * 2^32 + mid * 2^16 + lo (hi = v >> 32 signed, mid and lo
+// 16-bit) and the three parts are summed with 32-bit shared atomics: over
+// kKmUpdateRows rows the mid and lo sums stay below 2^27, and the hi sum below
+// 2^31 while the block's sum of |x| in one cluster stays below 2^23.  The
+// recombined total is exact, so neither the order of the atomics nor the
+// grouping into runs changes it.
 constexpr int kKmUpdateRows = 2048;
 
 template <int D>
 __global__ void __launch_bounds__(256) km_sum_kernel(const KmArgs a) {
-  extern __shared__ unsigned long long ss[];          // [C][D]
-  const int bh = blockIdx.y, C = a.C;
-  for (int i = threadIdx.x; i < C * D; i += blockDim.x) ss[i] = 0ull;
+  extern __shared__ uint32_t s32[];                   // [3][C][D]: hi, mid, lo
+  constexpr int E = D / 32;                           // dimensions per lane: lane + 32 e
+  constexpr int U = 4;                                // rows in flight per warp
+  const int bh = blockIdx.y, C = a.C, n = C * D;
+  uint32_t* s_hi = s32;
+  uint32_t* s_mid = s32 + n;
+  uint32_t* s_lo = s32 + 2 * n;
+  for (int i = threadIdx.x; i < 3 * n; i += blockDim.x) s32[i] = 0u;
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = blockDim.x >> 5;
   const int r0 = blockIdx.x * kKmUpdateRows, r1 = min(a.Lv, r0 + kKmUpdateRows);
-  for (int r = r0 + warp; r < r1; r += blockDim.x / 32) {
-    const int c = a.assign[static_cast<int64_t>(bh) * a.Lv + r];
-    const uint16_t* xr = a.x + (static_cast<int64_t>(bh) * a.L + r) * D;
-    for (int i = lane; i < D; i += 32) {
-      const double xv = static_cast<double>(__uint_as_float(static_cast<uint32_t>(xr[i]) << 16));
-      atomicAdd(&ss[c * D + i], static_cast<unsigned long long>(static_cast<long long>(xv * kFix)));
+  const int per = (r1 - r0 + nwarp - 1) / nwarp;
+  const int w0 = r0 + warp * per, w1 = min(r1, w0 + per);
+  const uint8_t* as = a.assign + static_cast<int64_t>(bh) * a.Lv;
+  const uint16_t* xh = a.x + static_cast<int64_t>(bh) * a.L * D;
+  long long acc[E];
+#pragma unroll
+  for (int e = 0; e < E; e++) acc[e] = 0;
+  int cur = -1;
+  auto flush = [&]() {
+    if (cur < 0) return;
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+      const int i = cur * D + lane + 32 * e;
+      const unsigned long long u = static_cast<unsigned long long>(acc[e]);
+      atomicAdd(&s_hi[i], static_cast<uint32_t>(static_cast<int32_t>(acc[e] >> 32)));
+      atomicAdd(&s_mid[i], static_cast<uint32_t>((u >> 16) & 0xFFFFu));
+      atomicAdd(&s_lo[i], static_cast<uint32_t>(u & 0xFFFFu));
+      acc[e] = 0;
+    }
+  };
+  for (int r = w0; r < w1; r += U) {
+    int cc[U];
+    uint16_t xv[U][E];
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int rr = r + u;
+      cc[u] = (rr < w1) ? static_cast<int>(__ldg(as + rr)) : -1;
+#pragma unroll
+      for (int e = 0; e < E; e++) xv[u][e] = (rr < w1) ? __ldg(xh + static_cast<int64_t>(rr) * D + lane + 32 * e) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      if (cc[u] < 0) continue;                        // warp-uniform: one row per step
+      if (cc[u] != cur) {
+        flush();
+        cur = cc[u];
+      }
+#pragma unroll
+      for (int e = 0; e < E; e++) {
+        const double xd = static_cast<double>(__uint_as_float(static_cast<uint32_t>(xv[u][e]) << 16));
+        acc[e] += static_cast<long long>(xd * kFix);
+      }
     }
   }
+  flush();
   __syncthreads();
-  unsigned long long* gs = a.sum + static_cast<int64_t>(bh) * C * D;
-  for (int i = threadIdx.x; i < C * D; i += blockDim.x)
-    if (ss[i]) atomicAdd(&gs[i], ss[i]);
+  unsigned long long* gs = a.sum + static_cast<int64_t>(bh) * n;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const long long hi = static_cast<int32_t>(s_hi[i]);
+    const unsigned long long t = (static_cast<unsigned long long>(hi) << 32) +
+                                 (static_cast<unsigned long long>(s_mid[i]) << 16) + s_lo[i];
+    if (t) atomicAdd(&gs[i], t);
+  }
 }
 
 // Means from the sums; clears the sums and the counts of the next assignment.

@@ -632,18 +632,18 @@ svg_status svg2_kmeans(const svg_shape* s, const uint16_t* x, int C, int iters, 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * a.BH * C, cs) != cudaSuccess) return SVG_ERR_CUDA;
   if (cudaMemsetAsync(workspace, 0, svg2_kmeans_workspace_size(s, C), cs) != cudaSuccess) return SVG_ERR_CUDA;
-  const dim3 cgrid(C, a.BH), agrid((Lv + 255) / 256, a.BH), sgrid((Lv + kKmUpdateRows - 1) / kKmUpdateRows, a.BH);
-  const int asmem = km_assign_pairs(C) * 2 * s->d * 4, ssmem = C * s->d * 8;
+  const dim3 cgrid(C, a.BH), agrid((Lv + kKmAssignRows - 1) / kKmAssignRows, a.BH), sgrid((Lv + kKmUpdateRows - 1) / kKmUpdateRows, a.BH);
+  const int asmem = km_assign_smem(C, s->d), ssmem = 3 * C * s->d * 4;
   auto run = [&](auto D_) -> svg_status {
     constexpr int D = decltype(D_)::value;
     if (!set_smem(km_assign_kernel<D>, asmem) || !set_smem(km_sum_kernel<D>, ssmem)) return SVG_ERR_CUDA;
     if (init) km_init_kernel<D><<<cgrid, D, 0, cs>>>(a);
     for (int t = 0; t < iters; t++) {
-      km_assign_kernel<D><<<agrid, 256, asmem, cs>>>(a);
+      km_assign_kernel<D><<<agrid, kKmAssignThreads, asmem, cs>>>(a);
       km_sum_kernel<D><<<sgrid, 256, ssmem, cs>>>(a);
       km_mean_kernel<D><<<cgrid, D, 0, cs>>>(a);
     }
-    km_assign_kernel<D><<<agrid, 256, asmem, cs>>>(a);
+    km_assign_kernel<D><<<agrid, kKmAssignThreads, asmem, cs>>>(a);
     return launch_status();
   };
   return s->d == 128 ? run(std::integral_constant<int, 128>{}) : run(std::integral_constant<int, 64>{});
