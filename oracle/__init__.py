@@ -23,6 +23,16 @@ Stages, with the page passages they follow (page title, section):
   describes needs it).
 * ``attention_rows`` -- masked softmax attention, the textbook definition.
 
+``svg2_oracle.c`` holds the semantic-aware permutation ("Sparse VideoGen2"
+explainer, "A. 语义感知排列", "B. 基于质心的 Top-p 选择"): ``kmeans`` (with
+``kmeans_init`` / ``kmeans_assign`` / ``kmeans_update``), ``cluster_permutation``,
+``select_top_p``, ``attention2_rows``, ``block_list2`` and ``permute_rows``.
+
+``adaspa_oracle.c`` holds AdaSpa's blockified search ("AdaSpa" abstract):
+``block_mass`` (exact block attention mass with a cached LSE),
+``adaspa_select`` (head-adaptive top-p over key tiles) and
+``block_attention_rows`` (attention over the kept tiles).
+
 Every function is pinned by ``tests/test_oracle_*.py``; none is "parity
 unpinned".
 """
@@ -38,6 +48,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "svg_oracle.c")
 _SRC2 = os.path.join(_HERE, "svg2_oracle.c")
+_SRC3 = os.path.join(_HERE, "adaspa_oracle.c")
 _BUILD = os.path.join(_HERE, "_build")
 _LIB = os.path.join(_BUILD, "liboracle.so")
 _lock = threading.Lock()
@@ -59,14 +70,14 @@ class OraParams(ctypes.Structure):
 
 
 def build(force: bool = False) -> str:
-    """Compile svg_oracle.c into oracle/_build/liboracle.so (gcc, -O2, OpenMP)."""
+    """Compile the oracle's C files into oracle/_build/liboracle.so (gcc, -O2, OpenMP)."""
     os.makedirs(_BUILD, exist_ok=True)
-    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC2))
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC2), os.path.getmtime(_SRC3))
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
         tmp = _LIB + f".tmp{os.getpid()}"
         # -std=c11 keeps a*b+c unfused (no contraction), as the oracle's text says
         subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-                               "-o", tmp, _SRC, _SRC2, "-lm"])
+                               "-o", tmp, _SRC, _SRC2, _SRC3, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -108,6 +119,11 @@ def lib():
                                               i64, vp, vp, vp]
             L.ora2_block_list.restype = i64
             L.ora2_block_list.argtypes = [ci, i64, i64, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp, vp, i64]
+            dbl = ctypes.c_double
+            L.ora3_block_mass.argtypes = [ci, i64, ci, ci, ci, dbl, vp, vp, vp, vp]
+            L.ora3_select.restype = i64
+            L.ora3_select.argtypes = [ci, i64, i64, ci, ci, vp, dbl, vp, vp, vp, i64]
+            L.ora3_attention_rows.argtypes = [ci, i64, ci, ci, ci, dbl, vp, vp, vp, vp, vp, i64, vp, vp, vp]
             _lib = L
     return _lib
 
@@ -377,3 +393,46 @@ def permute_rows(x, Lv: int, perm):
         for h in range(H):
             out[b, h, :Lv] = x[b, h, perm[b, h]]
     return out
+
+
+# ------------------------------------------------- AdaSpa blockified search --
+# "AdaSpa" abstract (blockified pattern; fused LSE-cached search; head-adaptive
+# hierarchical block sparse attention); the readings are stated at the top of
+# adaspa_oracle.c.
+
+def block_mass(q, k, lse, bq: int, bk: int, scale=None):
+    """fp64 block masses [BH, nqb, nkb] from bf16 q, k [B,H,L,d] and float lse [B,H,L]."""
+    q, k = _c(q, np.uint16), _c(k, np.uint16)
+    lse = _c(lse, np.float32)
+    BH, L, d = q.shape[0] * q.shape[1], q.shape[2], q.shape[3]
+    sc = 1.0 / np.sqrt(d) if scale is None else scale
+    nqb, nkb = -(-L // bq), -(-L // bk)
+    mass = np.empty((BH, nqb, nkb), np.float64)
+    lib().ora3_block_mass(BH, L, d, bq, bk, sc, _ptr(q), _ptr(k), _ptr(lse), _ptr(mass))
+    return mass
+
+
+def adaspa_select(mass, L: int, Lv: int, bq: int, bk: int, p: float):
+    """Kept key tiles from float32 masses [BH, nqb, nkb]: (row_ptr, col, full)."""
+    mass = _c(mass, np.float32)
+    BH, nqb, nkb = mass.shape
+    cap = BH * nqb * nkb
+    row_ptr = np.empty(BH * nqb + 1, np.int32)
+    col = np.empty(cap, np.int32)
+    full = np.empty(cap, np.uint8)
+    n = lib().ora3_select(BH, L, Lv, bq, bk, _ptr(mass), float(p), _ptr(row_ptr), _ptr(col), _ptr(full), cap)
+    return row_ptr, col[:n], full[:n]
+
+
+def block_attention_rows(q, k, v, bq: int, bk: int, row_ptr, col, rows, scale=None, want_lse=False):
+    """fp64 attention of `rows` (bh*L + token) over the kept key tiles of their query tile."""
+    q, k, v = (_c(t, np.uint16) for t in (q, k, v))
+    row_ptr, col = _c(row_ptr, np.int32), _c(col, np.int32)
+    rows = _c(rows, np.int64)
+    BH, L, d = q.shape[0] * q.shape[1], q.shape[2], q.shape[3]
+    sc = 1.0 / np.sqrt(d) if scale is None else scale
+    out = np.empty((len(rows), d), np.float64)
+    lse = np.empty(len(rows), np.float64) if want_lse else None
+    lib().ora3_attention_rows(BH, L, d, bq, bk, sc, _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), _ptr(col),
+                              len(rows), _ptr(rows), _ptr(out), _ptr(lse))
+    return (out, lse) if want_lse else out
