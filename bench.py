@@ -468,6 +468,116 @@ def run_svg2(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------- AdaSpa blockified search --
+
+def run_adaspa(args):
+    """AdaSpa's schedule on one GPU ("AdaSpa" abstract): a dense step caches
+    every row's LSE (untimed here: it is the last dense step of the schedule);
+    a search step computes the exact block masses under that LSE, picks the
+    kept tiles (top-p per head and query tile) and runs the block-sparse
+    attention; later steps reuse the pattern (attention only).  Prints one
+    JSON line; not the default bench line."""
+    import torch
+
+    import sparse_attention_video_qk_b200 as svg
+    from sparse_attention_video_qk_b200._lib import check
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    wl = W.WORKLOADS[args.workload]
+    pb = svg.Problem.from_workload(wl)
+    inp = W.make_inputs(wl)
+    q, k, v = (torch.from_numpy(inp[n]).view(torch.bfloat16).to(device) for n in ("q", "k", "v"))
+    gq, gk = (torch.from_numpy(inp[n]).to(device) for n in ("gamma_q", "gamma_k"))
+    table = torch.from_numpy(svg.rope_table(pb)).to(device)
+    qn, kn = svg.qknorm_rope(pb, q, k, gq, gk, table)
+    stream = torch.cuda.current_stream()
+    layer = svg.AdaSpaLayer(pb, args.adaspa_top_p)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    d0, d1 = ev(), ev()
+    layer.dense(qn, kn, v)
+    d0.record(stream)
+    layer.dense(qn, kn, v)                               # the cached LSE comes from this dense step
+    d1.record(stream)
+    mass = torch.empty(pb.B * pb.H, pb.nqb, pb.nkb, dtype=torch.float32, device=device)
+    cap = svg.block_index_capacity(pb)
+    rp = torch.empty(pb.B * pb.H * pb.nqb + 1, dtype=torch.int32, device=device)
+    col = torch.empty(cap, dtype=torch.int32, device=device)
+    full = torch.empty(cap, dtype=torch.uint8, device=device)
+    out = torch.empty_like(qn)
+    kinds = torch.full((pb.B * pb.H,), svg.DENSE, dtype=torch.uint8, device=device)
+    lib, sh, pr = svg.lib(), pb.c_shape(), pb.c_params()
+    cs = ctypes.c_void_p(stream.cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+
+    def search():
+        check(lib.svg_adaspa_block_mass(ctypes.byref(sh), ctypes.byref(pr), P(qn), P(kn), P(layer.lse),
+                                            P(mass), cs), "svg_adaspa_block_mass")
+
+    def select():
+        check(lib.svg_adaspa_select(ctypes.byref(sh), ctypes.byref(pr), P(mass), float(args.adaspa_top_p),
+                                        P(rp), P(col), P(full), cap, cs), "svg_adaspa_select")
+
+    def sparse():
+        check(lib.svg_block_sparse_attn(ctypes.byref(sh), ctypes.byref(pr), P(qn), P(kn), P(v), P(kinds),
+                                            P(rp), P(col), P(full), P(out), None, cs), "svg_block_sparse_attn")
+
+    for _ in range(args.warmup):
+        search()
+        select()
+        sparse()
+    svg.sync_status()
+    n_ent = int(rp[-1])
+    flops = kept_tile_flops(rp.cpu().numpy(), col[:n_ent].cpu().numpy(), wl)
+    evs = [[ev() for _ in range(4)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        clk.start()
+        for s_ in range(args.steps):
+            evs[s_][0].record(stream)
+            search()
+            evs[s_][1].record(stream)
+            select()
+            evs[s_][2].record(stream)
+            sparse()
+            evs[s_][3].record(stream)
+        torch.cuda.synchronize()
+        clk.stop()
+    svg.sync_status()
+    mean = lambda i: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+    mass_ms, select_ms, attn_ms = mean(0), mean(1), mean(2)
+    dense_ms = d0.elapsed_time(d1)
+    BH, L, d = wl.B * wl.H, wl.L, wl.d
+    pk, pk_src = peaks()
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    exps = float(BH) * L * L                               # one 2^x per (row, key)
+    mufu_peak = 148 * 16 * 1.965e9                         # 16 SFU results per SM per clock at 1965 MHz
+    line = {
+        "metric": "AdaSpa layer ms: search step (block masses + selection + sparse attention) and reuse step",
+        "value": round(mass_ms + select_ms + attn_ms, 3), "unit": "ms", "higher_is_better": False,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V with planted spatial/temporal heads; no model weights)",
+        "config": {"workload": f"{wl.name} ({SHAPE_LABEL[wl.name]}), AdaSpa blockified search",
+                   "top_p": args.adaspa_top_p, "tile": f"{wl.bq}x{wl.bk}",
+                   "tile_density": round(n_ent / (BH * wl.nqb * wl.nkb), 4),
+                   "kept_tile_tflop": round(flops / 1e12, 4)},
+        "stage_ms": {"block_mass": round(mass_ms, 3), "select": round(select_ms, 3), "attention": round(attn_ms, 3)},
+        "reuse_step_ms": round(attn_ms, 3),
+        "dense_attention_ms": round(dense_ms, 3),
+        "speedup_reuse_vs_dense": round(dense_ms / attn_ms, 3),
+        "roofline": {"kernel": f"attn2_kernel<{d}> (block list, every head dense)", "bound": "tensor",
+                     "achieved": round(attn_tflops, 2), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": round(attn_tflops / pk["bf16_tflops_sustained"], 4),
+                     "peak_source": f"{pk_src} bf16 sustained", "traffic": None},
+        "mass_roofline": {"kernel": f"mass_kernel<{d}>", "bound": "alu", "unit": "G exp2/s",
+                          "achieved": round(exps / (mass_ms * 1e-3) / 1e9, 1), "peak": round(mufu_peak / 1e9, 1),
+                          "frac": round(exps / (mass_ms * 1e-3) / mufu_peak, 4),
+                          "tensor_tflops": round(2.0 * BH * L * L * d / (mass_ms * 1e-3) / 1e12, 1)},
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------ sparsity sweep --
 
 def token_density(wl, kind):
@@ -664,6 +774,9 @@ def main():
     ap.add_argument("--svg2-clusters", type=int, default=64)
     ap.add_argument("--svg2-iters", type=int, default=2)
     ap.add_argument("--svg2-top-p", type=float, default=0.9)
+    ap.add_argument("--adaspa", action="store_true",
+                    help="time AdaSpa's search step and reuse step instead of the default step")
+    ap.add_argument("--adaspa-top-p", type=float, default=0.9)
     ap.add_argument("--sweep", action="store_true",
                     help="forced-kind sparsity sweep (one GPU); prints one JSON line with every point")
     args = ap.parse_args()
@@ -677,6 +790,10 @@ def main():
     if args.svg2:
         if rank == 0:
             run_svg2(args)
+        return
+    if args.adaspa:
+        if rank == 0:
+            run_adaspa(args)
         return
     if args.sweep:
         if rank == 0:

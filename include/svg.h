@@ -312,6 +312,39 @@ svg_status svg2_attention(const svg_shape* shape, const svg_params* params, cons
                           const uint64_t* sel, const int32_t* perm_q, const int32_t* row_ptr, const int32_t* col,
                           const uint8_t* full, uint16_t* out, float* lse_out, void* stream);
 
+/* --------------------------------------------- AdaSpa blockified search --
+ * "AdaSpa" abstract: a blockified sparse pattern, found by a "Fused
+ * LSE-Cached Search" and used by "Head-adaptive Hierarchical Block Sparse
+ * Attention"; the pattern and each row's log-sum-exp stay the same across
+ * denoising steps.  The search is exact given the cached LSE: the weight of a
+ * pair is exp(scale * q.k - lse_q), so one pass over Q K^T gives the mass of
+ * every (query tile, key tile) block.  The kept blocks then run through
+ * svg_block_sparse_attn with every head SVG_HEAD_DENSE (each listed block is
+ * computed whole).  Model order throughout; block_q = 128, block_k = 64. */
+
+/* Block masses.  q, k: device bf16 [B,H,L,d] (after QK-Norm + RoPE); lse:
+ * device float [B*H][L], the rows' natural log-sum-exp from an earlier step
+ * (e.g. the lse_out of a dense step of svg_block_sparse_attn); mass: device
+ * float [B*H][nqb][nkb]: mass[bh][qb][kb] = sum over rows q < L of tile qb and
+ * keys k < L of tile kb of exp(scale * q.k - lse[q]) (scores in fp32 on the
+ * tensor cores, 2^x by the hardware approximation, per-row sums in fp32, the
+ * tile's 128 rows added in a fixed order).  Requires block_q = 128, block_k = 64
+ * (SVG_ERR_UNSUPPORTED otherwise). */
+svg_status svg_adaspa_block_mass(const svg_shape* shape, const svg_params* params, const uint16_t* q,
+                                 const uint16_t* k, const float* lse, float* mass, void* stream);
+
+/* The kept key tiles of every (head, query tile), as CSR (same format as
+ * svg_build_block_index; every entry full = 1).  Video key tiles (no key in
+ * [Lv, L)) are ranked by mass, heavier first and the lower index on a tie; the
+ * shortest prefix whose running sum reaches top_p times their total is kept,
+ * at least one tile.  Sums are in 32-bit fixed point (mass * 2^32 truncated,
+ * exact in any order; the goal is top_p * total in double).  Key tiles holding
+ * text keys are always kept, and query tiles holding text rows keep every key
+ * tile.  mass: device float [B*H][nqb][nkb]; 0 < top_p <= 1; at most 4096 key
+ * tiles per query tile.  Capacity overflow is reported by svg_sync_status. */
+svg_status svg_adaspa_select(const svg_shape* shape, const svg_params* params, const float* mass, double top_p,
+                             int32_t* row_ptr, int32_t* col, uint8_t* full, int64_t capacity, void* stream);
+
 /* ----------------------------------------------------------- host helpers */
 
 /* n distinct video-token indices in [0, Lv) into host_out[0..n): the first n slots of

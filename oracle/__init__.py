@@ -120,7 +120,7 @@ def lib():
             L.ora2_block_list.restype = i64
             L.ora2_block_list.argtypes = [ci, i64, i64, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp, vp, i64]
             dbl = ctypes.c_double
-            L.ora3_block_mass.argtypes = [ci, i64, ci, ci, ci, dbl, vp, vp, vp, vp]
+            L.ora3_block_mass.argtypes = [ci, i64, ci, ci, ci, dbl, vp, vp, vp, i64, vp, vp]
             L.ora3_select.restype = i64
             L.ora3_select.argtypes = [ci, i64, i64, ci, ci, vp, dbl, vp, vp, vp, i64]
             L.ora3_attention_rows.argtypes = [ci, i64, ci, ci, ci, dbl, vp, vp, vp, vp, vp, i64, vp, vp, vp]
@@ -400,15 +400,22 @@ def permute_rows(x, Lv: int, perm):
 # hierarchical block sparse attention); the readings are stated at the top of
 # adaspa_oracle.c.
 
-def block_mass(q, k, lse, bq: int, bk: int, scale=None):
-    """fp64 block masses [BH, nqb, nkb] from bf16 q, k [B,H,L,d] and float lse [B,H,L]."""
+def block_mass(q, k, lse, bq: int, bk: int, scale=None, tiles=None):
+    """fp64 block masses [BH, nqb, nkb] from bf16 q, k [B,H,L,d] and float lse [B,H,L];
+    with `tiles` (ids bh*nqb + qb) only those query tiles, [len(tiles), nkb]."""
     q, k = _c(q, np.uint16), _c(k, np.uint16)
     lse = _c(lse, np.float32)
     BH, L, d = q.shape[0] * q.shape[1], q.shape[2], q.shape[3]
     sc = 1.0 / np.sqrt(d) if scale is None else scale
     nqb, nkb = -(-L // bq), -(-L // bk)
-    mass = np.empty((BH, nqb, nkb), np.float64)
-    lib().ora3_block_mass(BH, L, d, bq, bk, sc, _ptr(q), _ptr(k), _ptr(lse), _ptr(mass))
+    if tiles is None:
+        mass = np.empty((BH, nqb, nkb), np.float64)
+        lib().ora3_block_mass(BH, L, d, bq, bk, sc, _ptr(q), _ptr(k), _ptr(lse), 0, None, _ptr(mass))
+    else:
+        tiles = _c(tiles, np.int64)
+        mass = np.empty((len(tiles), nkb), np.float64)
+        lib().ora3_block_mass(BH, L, d, bq, bk, sc, _ptr(q), _ptr(k), _ptr(lse), len(tiles), _ptr(tiles),
+                              _ptr(mass))
     return mass
 
 

@@ -43,18 +43,21 @@ static double bf16_to_f64_3(uint16_t h) {
 
 #define ORA3_FIX 4294967296.0 /* 2^32 */
 
-/* Block masses.  Q, K: bf16 [BH][L][d]; lse: float [BH][L] (natural log);
- * mass: double [BH][nqb][nkb], nqb = ceil(L / bq), nkb = ceil(L / bk).
+/* Block masses.  Q, K: bf16 [BH][L][d]; lse: float [BH][L] (natural log).
  * mass[bh][qb][kb] = sum over rows q < L of tile qb and keys k < L of tile kb
- * of exp(scale * q.k - lse[q]). */
+ * of exp(scale * q.k - lse[q]), nqb = ceil(L / bq), nkb = ceil(L / bk).
+ * With tiles == NULL, mass is double [BH][nqb][nkb]; otherwise only the
+ * ntiles query tiles tiles[i] = bh * nqb + qb, into mass [ntiles][nkb]. */
 void ora3_block_mass(int BH, int64_t L, int d, int bq, int bk, double scale, const uint16_t* Q,
-                     const uint16_t* K, const float* lse, double* mass) {
+                     const uint16_t* K, const float* lse, int64_t ntiles, const int64_t* tiles, double* mass) {
   int64_t nqb = (L + bq - 1) / bq, nkb = (L + bk - 1) / bk;
-  memset(mass, 0, sizeof(double) * (size_t)BH * nqb * nkb);
+  int64_t nt = tiles ? ntiles : (int64_t)BH * nqb;
+  memset(mass, 0, sizeof(double) * (size_t)nt * nkb);
 #pragma omp parallel for schedule(dynamic, 1)
-  for (int64_t t = 0; t < (int64_t)BH * nqb; t++) {
+  for (int64_t i = 0; i < nt; i++) {
+    int64_t t = tiles ? tiles[i] : i;
     int64_t bh = t / nqb, qb = t % nqb;
-    double* m = mass + t * nkb;
+    double* m = mass + i * nkb;
     for (int64_t q = qb * bq; q < (qb + 1) * bq && q < L; q++) {
       const uint16_t* qr = Q + (bh * L + q) * d;
       double lq = (double)lse[bh * L + q];

@@ -479,6 +479,71 @@ class SVG2Layer:
         return out
 
 
+# ---------------------------------------------- AdaSpa blockified search --
+
+def adaspa_block_mass(pb: Problem, q, k, lse, out=None, stream=None):
+    """Block attention masses float [B*H, nqb, nkb] from normalised q, k (bf16
+    [B,H,L,d]) and each row's cached log-sum-exp (float [B,H,L])."""
+    sh, pr = pb.c_shape(), pb.c_params()
+    if out is None:
+        out = torch.empty(pb.B * pb.H, pb.nqb, pb.nkb, dtype=torch.float32, device=q.device)
+    check(lib().svg_adaspa_block_mass(ctypes.byref(sh), ctypes.byref(pr), _p(q), _p(k), _p(lse), _p(out),
+                                      _stream(stream)), "svg_adaspa_block_mass")
+    return out
+
+
+def adaspa_select(pb: Problem, mass, top_p: float, capacity=None, stream=None):
+    """Kept key tiles (row_ptr, col, full) of every (head, query tile)."""
+    sh, pr = pb.c_shape(), pb.c_params()
+    if capacity is None:
+        capacity = block_index_capacity(pb)
+    dev = mass.device
+    row_ptr = torch.empty(pb.B * pb.H * pb.nqb + 1, dtype=torch.int32, device=dev)
+    col = torch.empty(capacity, dtype=torch.int32, device=dev)
+    full = torch.empty(capacity, dtype=torch.uint8, device=dev)
+    check(lib().svg_adaspa_select(ctypes.byref(sh), ctypes.byref(pr), _p(mass), float(top_p), _p(row_ptr), _p(col),
+                                  _p(full), capacity, _stream(stream)), "svg_adaspa_select")
+    return row_ptr, col, full
+
+
+class AdaSpaLayer:
+    """AdaSpa's schedule for one layer: a dense step keeps every row's LSE;
+    at a search step the block masses under that cached LSE pick the kept
+    tiles (top-p per head and query tile); later steps reuse the pattern
+    until the next search.  Works on normalised Q, K (model order)."""
+
+    def __init__(self, pb: Problem, top_p: float = 0.9):
+        self.pb, self.top_p = pb, top_p
+        self.lse = None
+        self.blocks = None
+        self._dense_kinds = None
+
+    def _kinds(self, device):
+        if self._dense_kinds is None or self._dense_kinds.device != device:
+            self._dense_kinds = torch.full((self.pb.B * self.pb.H,), DENSE, dtype=torch.uint8, device=device)
+        return self._dense_kinds
+
+    def dense(self, qn, kn, v, stream=None):
+        """Dense attention; keeps each row's LSE for the next search."""
+        kinds = self._kinds(qn.device)
+        rp, col, full = build_block_index(self.pb, kinds, stream=stream)
+        out, self.lse = block_sparse_attn(self.pb, qn, kn, v, kinds, rp, col, full, want_lse=True, stream=stream)
+        return out
+
+    def search(self, qn, kn, stream=None):
+        if self.lse is None:
+            raise RuntimeError("AdaSpaLayer.search needs the LSE of an earlier dense step")
+        mass = adaspa_block_mass(self.pb, qn, kn, self.lse, stream=stream)
+        self.blocks = adaspa_select(self.pb, mass, self.top_p, stream=stream)
+        return mass
+
+    def sparse(self, qn, kn, v, stream=None):
+        if self.blocks is None:
+            raise RuntimeError("AdaSpaLayer.sparse needs a search first")
+        rp, col, full = self.blocks
+        return block_sparse_attn(self.pb, qn, kn, v, self._kinds(qn.device), rp, col, full, stream=stream)
+
+
 # ------------------------------------------------------ denoising schedule --
 
 STEP_DENSE, STEP_PROFILE, STEP_REUSE = C.SVG_STEP_DENSE, C.SVG_STEP_PROFILE, C.SVG_STEP_REUSE

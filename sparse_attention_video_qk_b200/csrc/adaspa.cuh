@@ -1,0 +1,420 @@
+// adaspa.cuh — AdaSpa's blockified search with a cached LSE ("AdaSpa"
+// abstract: a blockified sparse pattern; "Fused LSE-Cached Search with
+// Head-adaptive Hierarchical Block Sparse Attention"; the pattern and the LSE
+// stay the same across denoising steps).
+//
+// 1. mass_kernel: the exact attention mass of every (query tile, key tile)
+//    block, given each row's log-sum-exp from an earlier step:
+//        M[qb][kb] = sum_{q in qb, k in kb} 2^(s_qk * scale * log2 e - lse_q * log2 e)
+//    in one pass over Q K^T (no normalisation pass: the LSE is known).  The
+//    CTA layout follows the attention kernel: one CTA per (b, h, pair of
+//    128-row query tiles), warp 0 streams K through a TMA slot ring, warp 1
+//    issues S = Q K^T as M=128, N=128 tcgen05 MMAs into TMEM, warps 2-5 and
+//    6-9 exponentiate and sum the two query tiles' S (thread = row).  S is
+//    double-buffered per query tile (4 x 128 TMEM columns), so the MMAs of
+//    tile j+1 overlap the exponentials of tile j.  The per-row sums of each
+//    64-key block are reduced over the tile's 128 rows by shuffles and a fixed
+//    4-warp order, so the result does not depend on scheduling.
+// 2. select_kernel: per (head, query tile), the video key tiles sorted by
+//    mass (descending, lower index first) and the shortest prefix whose
+//    running sum reaches p times their total, in 32-bit fixed point; text key
+//    tiles always, and query tiles holding text rows keep every key tile.
+//    One block per query tile: bitonic sort in shared memory, a block scan of
+//    the fixed-point masses, then the kept tiles in increasing order.
+//
+// Every mbarrier wait is bounded; on time-out the kernel records
+// kErrTimeout, drains its outstanding copies and MMAs, frees TMEM and returns.
+#pragma once
+
+#include "attention.cuh"
+#include "svg_common.cuh"
+
+namespace svg {
+
+template <int D>
+struct MassCfg {
+  static constexpr int PANELS = D / 64;
+  static constexpr int PANEL = 128 * 128;          // bytes of one 128-row panel
+  static constexpr int Q_BYTES = 128 * D * 2;      // one query tile
+  static constexpr int SLOT_BYTES = 128 * D * 2;   // one 128-key K tile
+  static constexpr int NSLOT = (D == 128) ? 4 : 8;
+  static constexpr int DATA_BYTES = 2 * Q_BYTES + NSLOT * SLOT_BYTES;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMEM_BYTES = DATA_BYTES + BAR_BYTES + 1024;
+  static constexpr int THREADS = 320;
+  static constexpr uint32_t TMEM_COLS = 512;
+  // TMEM columns: S of query tile w, buffer b at 256*w + 128*b
+  static __device__ __forceinline__ uint32_t tm_s(int w, int b) { return 256u * w + 128u * b; }
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(20 + 2 * NSLOT + 16 <= BAR_BYTES / 8, "barrier area");
+};
+
+struct MassArgs {
+  Geometry g;
+  float scale_log2;        // softmax scale * log2(e)
+  const float* lse;        // [BH][L], natural log, cached from an earlier step
+  float* mass;             // [BH][nqb][nkb]
+};
+
+template <int D>
+__global__ void __launch_bounds__(MassCfg<D>::THREADS, 1)
+    mass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                const MassArgs a) {
+  using C = MassCfg<D>;
+  constexpr int NSLOT = C::NSLOT;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + 2 * C::Q_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::DATA_BYTES);
+  // barriers: q | full[NSLOT] | empty[NSLOT] | s[2][2] | free[2][2] | part[2][2] | pfree[2][2] |
+  // drain; then the TMEM slot, the abort flag and the per-warp partial sums
+  const uint32_t b_q = smem_addr(&bars[0]);
+  auto b_full = [&](int s) { return smem_addr(&bars[1 + s]); };
+  auto b_empty = [&](int s) { return smem_addr(&bars[1 + NSLOT + s]); };
+  auto b_s = [&](int w, int b) { return smem_addr(&bars[1 + 2 * NSLOT + 2 * w + b]); };
+  auto b_free = [&](int w, int b) { return smem_addr(&bars[5 + 2 * NSLOT + 2 * w + b]); };
+  auto b_part = [&](int w, int b) { return smem_addr(&bars[9 + 2 * NSLOT + 2 * w + b]); };
+  auto b_pfree = [&](int w, int b) { return smem_addr(&bars[13 + 2 * NSLOT + 2 * w + b]); };
+  const uint32_t b_drain = smem_addr(&bars[17 + 2 * NSLOT]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[18 + 2 * NSLOT]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[19 + 2 * NSLOT]);
+  float* part = reinterpret_cast<float*>(&bars[20 + 2 * NSLOT]);   // [2 groups][2 bufs][4 warps][2]
+
+  const Geometry& g = a.g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int npair = (g.nqb + 1) >> 1;
+  const int bh = blockIdx.x / npair, qb0 = 2 * (blockIdx.x % npair);
+  const int ntile = (g.nkb + 1) >> 1;                  // 128-key tiles: blocks 2j, 2j+1
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_q, 1);
+    for (int s = 0; s < NSLOT; s++) {
+      mbar_init(b_full(s), 1);
+      mbar_init(b_empty(s), 1);
+    }
+    for (int w = 0; w < 2; w++)
+      for (int b = 0; b < 2; b++) {
+        mbar_init(b_s(w, b), 1);
+        mbar_init(b_free(w, b), 128);
+        mbar_init(b_part(w, b), 4);
+        mbar_init(b_pfree(w, b), 1);
+      }
+    mbar_init(b_drain, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmq);
+      tma_prefetch_desc(&tmk);
+      mbar_expect_tx(b_q, 2 * C::Q_BYTES);
+#pragma unroll
+      for (int w = 0; w < 2; w++)
+#pragma unroll
+        for (int p = 0; p < C::PANELS; p++)
+          tma_load_3d(smem_addr(sQ + w * C::Q_BYTES + p * C::PANEL), &tmq, p * 64, (qb0 + w) * 128, bh, b_q);
+      int issued = 0;
+      for (int j = 0; j < ntile; j++) {
+        const int st = j % NSLOT;
+        if (j >= NSLOT && !mbar_wait(b_empty(st), ((j / NSLOT) - 1) & 1, abort_flag)) break;
+        const int nb = (2 * j + 1 < g.nkb) ? 2 : 1;
+        mbar_expect_tx(b_full(st), nb * 64 * D * 2);
+        for (int h = 0; h < nb; h++)
+#pragma unroll
+          for (int p = 0; p < C::PANELS; p++)
+            tma_load_3d(smem_addr(sK + st * C::SLOT_BYTES + p * C::PANEL + h * 64 * 128), &tmk, p * 64,
+                        (2 * j + h) * 64, bh, b_full(st));
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait_drain(b_q, 0);
+        for (int i = max(0, issued - NSLOT); i < issued; i++) mbar_wait_drain(b_full(i % NSLOT), (i / NSLOT) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS128 = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idS64 = idesc_bf16_f32(128, 64, 0, 0);
+      const uint32_t q_base = smem_addr(sQ), k_base = smem_addr(sK);
+      bool issued_any = false;
+      bool ok = mbar_wait(b_q, 0, abort_flag);
+      for (int j = 0; ok && j < ntile; j++) {
+        const int st = j % NSLOT, b = j & 1;
+        const int nb = (2 * j + 1 < g.nkb) ? 2 : 1;
+        if (!mbar_wait(b_full(st), (j / NSLOT) & 1, abort_flag)) break;
+        for (int w = 0; w < 2 && ok; w++) {
+          // S_w buffer b was last read by the softmax at tile j-2
+          if (j >= 2 && !mbar_wait(b_free(w, b), ((j >> 1) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; kk++) {
+            const uint32_t off = (kk >> 2) * C::PANEL + (kk & 3) * 32;
+            umma_ss(tmem + C::tm_s(w, b), sdesc_sw128(q_base + w * C::Q_BYTES + off, 16, 1024),
+                    sdesc_sw128(k_base + st * C::SLOT_BYTES + off, 16, 1024), nb == 2 ? idS128 : idS64, kk > 0);
+          }
+          umma_commit(b_s(w, b));
+          issued_any = true;
+        }
+        if (!ok) break;
+        umma_commit(b_empty(st));
+      }
+      if (*abort_flag && issued_any) {
+        umma_commit(b_drain);
+        mbar_wait_drain(b_drain, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ exponentials (two groups)
+    const int w = (warp - 2) >> 2;                 // query tile of this group
+    const int q4 = warp & 3;                       // TMEM lane quarter
+    const int wg = (warp - 2) & 3;                 // warp index inside the group
+    const int r = q4 * 32 + lane;
+    const int row = (qb0 + w) * 128 + r;
+    const bool tile_ok = (qb0 + w) < g.nqb;
+    // rows past L contribute nothing: 2^(s - inf) = 0
+    const float l2 = (row < g.L) ? __ldg(a.lse + static_cast<int64_t>(bh) * g.L + row) * 1.4426950408889634f
+                                 : INFINITY;
+    const uint64_t sl2x2 = f32x2(a.scale_log2, a.scale_log2);
+    const uint64_t nl2x2 = f32x2(-l2, -l2);
+    const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    float* mrow = a.mass + (static_cast<int64_t>(bh) * g.nqb + qb0 + w) * g.nkb;
+    for (int j = 0; j < ntile; j++) {
+      const int b = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(b_s(w, b), (j >> 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t tS = tl + C::tm_s(w, b);
+      float h[2];
+#pragma unroll
+      for (int half = 0; half < 2; half++) {
+        const int kb = 2 * j + half;
+        uint64_t acc[2] = {0ull, 0ull};
+        if (kb < g.nkb) {                          // warp-uniform
+#pragma unroll
+          for (int q = 0; q < 2; q++) {
+            uint32_t v[32];
+            tmem_ld32(tS + half * 64 + q * 32, v);
+            tmem_wait_ld();
+            const int k0 = kb * 64 + q * 32;
+            if (k0 + 32 > g.L) {                   // the ragged last block: keys past L hold zero rows
+#pragma unroll
+              for (int c = 0; c < 32; c++)
+                if (k0 + c >= g.L) v[c] = __float_as_uint(-INFINITY);
+            }
+#pragma unroll
+            for (int c = 0; c < 16; c++) {
+              const uint64_t x = ffma2(f32x2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])), sl2x2, nl2x2);
+              float x0, x1;
+              unpack2(x, x0, x1);
+              acc[c & 1] = fadd2(acc[c & 1], f32x2(fast_exp2(x0), fast_exp2(x1)));
+            }
+          }
+        }
+        float s0, s1, s2, s3;
+        unpack2(acc[0], s0, s1);
+        unpack2(acc[1], s2, s3);
+        h[half] = (s0 + s1) + (s2 + s3);
+      }
+      tc_fence_before();
+      mbar_arrive(b_free(w, b));
+      // the block sums of this tile over the group's 128 rows: shuffles inside a
+      // warp, then the group's first warp adds the four warps in a fixed order.
+      // The hand-off goes through mbarriers (bounded waits), double-buffered
+      // like S: part(w, b) completes when the four warps have written, pfree(w, b)
+      // when the first warp has read them.
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        h[0] += __shfl_xor_sync(0xffffffffu, h[0], o);
+        h[1] += __shfl_xor_sync(0xffffffffu, h[1], o);
+      }
+      float* pb = part + ((w * 2 + b) * 4) * 2;
+      int okp = 1;
+      if (lane == 0) {
+        if (j >= 2) okp = mbar_wait(b_pfree(w, b), ((j >> 1) - 1) & 1, abort_flag);
+        if (okp) {
+          pb[wg * 2] = h[0];
+          pb[wg * 2 + 1] = h[1];
+          mbar_arrive(b_part(w, b));
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, okp, 0)) break;
+      if (wg == 0) {
+        int okr = 1;
+        if (lane == 0) {
+          okr = mbar_wait(b_part(w, b), (j >> 1) & 1, abort_flag);
+          if (okr) {
+            const float m0 = ((pb[0] + pb[2]) + pb[4]) + pb[6];
+            const float m1 = ((pb[1] + pb[3]) + pb[5]) + pb[7];
+            mbar_arrive(b_pfree(w, b));
+            if (tile_ok) {
+              mrow[2 * j] = m0;
+              if (2 * j + 1 < g.nkb) mrow[2 * j + 1] = m1;
+            }
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, okr, 0)) break;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ selection
+
+struct SelArgs {
+  Geometry g;
+  double p;
+  const float* mass;       // [BH][nqb][nkb]
+};
+
+constexpr int kSelThreads = 1024;
+constexpr int kSelMaxTiles = 4096;         // key tiles per query tile (L <= 262,144 at bk = 64)
+
+__device__ __forceinline__ bool sel_before(float ma, int ia, float mb, int ib) {
+  return (ma > mb) || (ma == mb && ia < ib);
+}
+
+// Block-wide inclusive scan of one int64 per thread (kSelThreads threads).
+__device__ __forceinline__ long long sel_block_scan(long long v, long long* warp_tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  if (lane == 31) warp_tot[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    long long t = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long u = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += u;
+    }
+    warp_tot[lane] = t;
+  }
+  __syncthreads();
+  const long long base = warp ? warp_tot[warp - 1] : 0;
+  __syncthreads();
+  return v + base;
+}
+
+// FILL = false: row_ptr[t + 1] = number of kept tiles; FILL = true: the kept
+// tiles in increasing order at col[row_ptr[t] ...], full = 1.
+template <bool FILL>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a, int32_t* __restrict__ row_ptr,
+                                                            int32_t* __restrict__ col, uint8_t* __restrict__ full,
+                                                            int64_t capacity, int P2) {
+  extern __shared__ uint8_t sel_smem[];
+  float* sm = reinterpret_cast<float*>(sel_smem);              // [P2] masses, sorted in place
+  int* si = reinterpret_cast<int*>(sm + P2);                    // [P2] tile indices
+  uint8_t* keep = reinterpret_cast<uint8_t*>(si + P2);          // [P2] kept flags by tile index
+  __shared__ long long warp_tot[32];
+  __shared__ int s_cut;
+  const Geometry& g = a.g;
+  const int64_t t = blockIdx.x;                                 // bh * nqb + qb
+  const int qb = static_cast<int>(t % g.nqb);
+  const int tid = threadIdx.x;
+  const float* m = a.mass + t * g.nkb;
+  const bool text_q = min(g.L, (qb + 1) * g.bq) > g.Lv;
+  // video key tiles: no key in [Lv, L) (without text, every tile)
+  const int nv = (g.L == g.Lv) ? g.nkb : min(g.nkb, g.Lv / g.bk);
+  for (int i = tid; i < P2; i += kSelThreads) {
+    const bool vid = i < nv;
+    sm[i] = vid ? __ldg(m + i) : -INFINITY;
+    si[i] = i;
+    keep[i] = (i < g.nkb && (text_q || !vid)) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!text_q && nv > 0) {
+    // bitonic sort of (mass, index): heavier first, the lower index first on ties
+    for (int k = 2; k <= P2; k <<= 1)
+      for (int jj = k >> 1; jj > 0; jj >>= 1) {
+        for (int i = tid; i < P2; i += kSelThreads) {
+          const int l = i ^ jj;
+          if (l > i) {
+            const bool up = (i & k) == 0;
+            const float ma = sm[i], mb = sm[l];
+            const int ia = si[i], ib = si[l];
+            const bool swap = up ? sel_before(mb, ib, ma, ia) : sel_before(ma, ia, mb, ib);
+            if (swap) {
+              sm[i] = mb;
+              sm[l] = ma;
+              si[i] = ib;
+              si[l] = ia;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    // fixed-point masses in sorted order: each thread owns P2 / kSelThreads consecutive positions
+    const int per = P2 / kSelThreads > 0 ? P2 / kSelThreads : 1;
+    const int p0 = tid * per;
+    long long own = 0;
+    for (int u = 0; u < per; u++) {
+      const int pos = p0 + u;
+      if (pos < nv) own += static_cast<long long>(static_cast<double>(sm[pos]) * 4294967296.0);
+    }
+    const long long incl = sel_block_scan(own, warp_tot);
+    const long long total = warp_tot[31];
+    const double goal = __dmul_rn(a.p, static_cast<double>(total));
+    // positions whose inclusive running sum is still below the goal
+    long long run = incl - own;
+    int below = 0;
+    for (int u = 0; u < per; u++) {
+      const int pos = p0 + u;
+      if (pos < nv) {
+        run += static_cast<long long>(static_cast<double>(sm[pos]) * 4294967296.0);
+        below += (static_cast<double>(run) < goal) ? 1 : 0;
+      }
+    }
+    if (tid == 0) s_cut = 0;
+    __syncthreads();
+    if (below) atomicAdd(&s_cut, below);
+    __syncthreads();
+    const int cut = s_cut;                                      // positions 0..cut are kept
+    for (int pos = tid; pos <= cut && pos < nv; pos += kSelThreads) keep[si[pos]] = 1;
+    __syncthreads();
+  }
+  // the kept tiles in increasing order
+  const int per = (g.nkb + kSelThreads - 1) / kSelThreads;
+  const int i0 = tid * per;
+  int cnt = 0;
+  for (int u = 0; u < per; u++)
+    if (i0 + u < g.nkb) cnt += keep[i0 + u];
+  const long long incl = sel_block_scan(cnt, warp_tot);
+  if (!FILL) {
+    if (tid == kSelThreads - 1) row_ptr[t + 1] = static_cast<int32_t>(incl);
+    if (t == 0 && tid == 0) row_ptr[0] = 0;
+    return;
+  }
+  int64_t e = row_ptr[t] + (incl - cnt);
+  for (int u = 0; u < per; u++) {
+    const int kb = i0 + u;
+    if (kb < g.nkb && keep[kb]) {
+      if (e < capacity) {
+        col[e] = kb;
+        full[e] = 1;
+      }
+      e++;
+    }
+  }
+}
+
+}  // namespace svg

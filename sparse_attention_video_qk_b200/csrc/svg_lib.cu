@@ -16,6 +16,7 @@
 #include "profile_tc.cuh"
 #include "rowmap.cuh"
 #include "svg2.cuh"
+#include "adaspa.cuh"
 #include "svg_common.cuh"
 
 using namespace svg;
@@ -753,6 +754,60 @@ svg_status svg2_attention(const svg_shape* s, const svg_params* p, const uint16_
   c.Ck = Ck;
   c.out_perm = perm_q;
   return attention_launch(s, p, q, k, v, nullptr, row_ptr, col, full, out, lse_out, 0, stream, &c);
+}
+
+// ------------------------------------------------ AdaSpa blockified search
+
+svg_status svg_adaspa_block_mass(const svg_shape* s, const svg_params* p, const uint16_t* q, const uint16_t* k,
+                                 const float* lse, float* mass, void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if ((st = check_params(s, p, true)) != SVG_OK) return st;
+  if (!q || !k || !lse || !mass) return SVG_ERR_INVALID_ARG;
+  if (p->block_q != 128 || p->block_k != 64) return SVG_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return SVG_ERR_ALIGNMENT;
+  MassArgs a{};
+  a.g = make_geometry(s, p);
+  a.scale_log2 = scale_of(s, p) * 1.4426950408889634f;
+  a.lse = lse;
+  a.mass = mass;
+  CUtensorMap mq, mk;
+  if (!make_map(&mq, q, s->d, s->L, a.g.BH, 128) || !make_map(&mk, k, s->d, s->L, a.g.BH, 64)) return SVG_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(a.g.BH) * static_cast<unsigned>((a.g.nqb + 1) / 2);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  auto run = [&](auto kern, int smem) -> svg_status {
+    if (!set_smem(kern, smem)) return SVG_ERR_CUDA;
+    kern<<<grid, MassCfg<128>::THREADS, smem, cs>>>(mq, mk, a);
+    return launch_status();
+  };
+  return s->d == 128 ? run(mass_kernel<128>, MassCfg<128>::SMEM_BYTES) : run(mass_kernel<64>, MassCfg<64>::SMEM_BYTES);
+}
+
+svg_status svg_adaspa_select(const svg_shape* s, const svg_params* p, const float* mass, double top_p,
+                             int32_t* row_ptr, int32_t* col, uint8_t* full, int64_t capacity, void* stream) {
+  svg_status st = check_shape(s);
+  if (st != SVG_OK) return st;
+  if ((st = check_params(s, p, true)) != SVG_OK) return st;
+  if (!mass || !row_ptr || !col || !full || capacity < 0) return SVG_ERR_INVALID_ARG;
+  if (!(top_p > 0.0) || !(top_p <= 1.0)) return SVG_ERR_INVALID_ARG;
+  SelArgs a{};
+  a.g = make_geometry(s, p);
+  a.p = top_p;
+  a.mass = mass;
+  if (a.g.nkb > kSelMaxTiles) return SVG_ERR_UNSUPPORTED;
+  int P2 = 2;
+  while (P2 < a.g.nkb) P2 <<= 1;
+  const int smem = P2 * 9;
+  const int64_t n = static_cast<int64_t>(a.g.BH) * a.g.nqb;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  select_kernel<false><<<static_cast<unsigned>(n), kSelThreads, smem, cs>>>(a, row_ptr, col, full, capacity, P2);
+  if ((st = launch_status()) != SVG_OK) return st;
+  block_scan_kernel<<<1, 1024, 0, cs>>>(row_ptr, n, capacity);
+  if ((st = launch_status()) != SVG_OK) return st;
+  select_kernel<true><<<static_cast<unsigned>(n), kSelThreads, smem, cs>>>(a, row_ptr, col, full, capacity, P2);
+  return launch_status();
 }
 
 }  // extern "C"

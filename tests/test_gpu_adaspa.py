@@ -1,0 +1,259 @@
+"""Parity of AdaSpa's blockified LSE-cached search ("AdaSpa" abstract) with
+the oracle, through the C ABI.
+
+Bars:
+  * block masses: |gpu - oracle| <= 2e-4 * oracle + 1e-6 * (rows of the tile)
+    (fp32 scores on the tensor cores, the hardware 2^x, fp32 sums);
+  * selection on the same float masses: bit-exact CSR;
+  * attention over a block list: max-abs 2e-2, mean-abs 2e-3 against fp64;
+  * the whole search on the GPU: its selection equals the oracle's on every
+    query tile whose decision is clear of the mass tolerance.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_attention_video_qk_b200 as svg
+import svg_workloads as W
+from gpu_util import assert_attention_close, dev, host_bits
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # d = 128, text, ragged last key tile (L = 403 = 6 * 64 + 19), 4 query tiles
+    "d128": (W.small_workload(d=128, H=2, F=4, Hs=8, Ws=12, T=19, seed=31), 0.9),
+    # d = 64, three heads, an odd number of query tiles (the last pair has one)
+    "d64": (W.small_workload(d=64, H=3, F=5, Hs=6, Ws=10, T=7, seed=32), 0.8),
+    # no text, Lv not a multiple of 64: the ragged last key tile is a video tile
+    "notext": (W.small_workload(d=128, H=2, F=3, Hs=7, Ws=9, T=0, seed=33), 0.95),
+    # two batch entries
+    "batch2": (W.small_workload(B=2, d=128, H=2, F=3, Hs=8, Ws=8, T=5, seed=34), 0.7),
+    # Wan 2.1 1.3B shape (sampled query tiles)
+    "wan": (W.WAN, 0.9),
+}
+SMALL = ("d128", "d64", "notext", "batch2")
+
+
+def pb_of(wl):
+    return svg.Problem.from_workload(wl)
+
+
+def dense_lse(qn, kn, wl, tiles=None):
+    """Each row's log-sum-exp over all keys (fp64 numpy, rounded to float):
+    the LSE a dense step would cache.  With `tiles`, only the rows of those
+    query tiles; the other rows get log(L)."""
+    BH, L, d = wl.B * wl.H, wl.L, wl.d
+    q = W.bf16_bits_to_f32(qn.reshape(BH, L, d)).astype(np.float64)
+    k = W.bf16_bits_to_f32(kn.reshape(BH, L, d)).astype(np.float64)
+    lse = np.full((BH, L), np.log(L), np.float64)
+    todo = range(BH * wl.nqb) if tiles is None else tiles
+    for t in todo:
+        bh, qb = divmod(int(t), wl.nqb)
+        r0, r1 = qb * wl.bq, min(L, (qb + 1) * wl.bq)
+        s = q[bh, r0:r1] @ k[bh].T / np.sqrt(d)
+        m = s.max(1, keepdims=True)
+        lse[bh, r0:r1] = m[:, 0] + np.log(np.exp(s - m).sum(1))
+    return lse.astype(np.float32).reshape(wl.B, wl.H, L)
+
+
+@functools.lru_cache(maxsize=None)
+def case(key):
+    wl, p = CASES[key]
+    inp = W.make_inputs(wl)
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    qn = oracle.qknorm_rope(sh, pr, inp["q"], inp["gamma_q"])
+    kn = oracle.qknorm_rope(sh, pr, inp["k"], inp["gamma_k"])
+    if key in SMALL:
+        tiles = None
+    else:
+        rng = np.random.Generator(np.random.PCG64(5))
+        tiles = np.sort(rng.choice(wl.B * wl.H * wl.nqb, 12, replace=False)).astype(np.int64)
+        # the last query tile of head 0 holds the text rows and the ragged tail
+        tiles = np.unique(np.concatenate([tiles, [wl.nqb - 1]])).astype(np.int64)
+    lse = dense_lse(qn, kn, wl, tiles)
+    mass = oracle.block_mass(qn, kn, lse, wl.bq, wl.bk, tiles=tiles)
+    return wl, p, inp, qn, kn, lse, tiles, mass
+
+
+def rows_in_tiles(wl, tiles):
+    q = np.arange(wl.nqb * wl.bq)
+    out = []
+    for t in tiles:
+        bh, qb = divmod(int(t), wl.nqb)
+        r = q[qb * wl.bq:(qb + 1) * wl.bq]
+        out.append(r[r < wl.L])
+    return np.concatenate(out), np.repeat(np.arange(len(tiles)), [len(x) for x in out])
+
+
+@pytest.mark.parametrize("key", list(CASES))
+def test_block_mass_against_fp64(key):
+    wl, p, inp, qn, kn, lse, tiles, want = case(key)
+    got = svg.adaspa_block_mass(pb_of(wl), dev(qn), dev(kn), dev(lse))
+    svg.sync_status()
+    got = got.cpu().numpy().reshape(-1, wl.nkb).astype(np.float64)
+    if tiles is not None:
+        got = got[tiles]
+    want = want.reshape(-1, wl.nkb)
+    err = np.abs(got - want)
+    bound = 2e-4 * want + 1e-6 * wl.bq
+    assert (err <= bound).all(), f"{key}: worst excess {(err - bound).max():.3e}"
+    if tiles is None:
+        # with the exact LSE every row's weights sum to 1
+        rows = np.minimum(wl.bq, wl.L - np.arange(wl.nqb) * wl.bq)
+        assert np.allclose(got.reshape(-1, wl.nqb, wl.nkb).sum(-1), rows[None, :], rtol=1e-3)
+
+
+@pytest.mark.parametrize("key", SMALL)
+def test_select_bit_exact_on_the_same_masses(key):
+    wl, p, inp, qn, kn, lse, tiles, mass = case(key)
+    m32 = mass.astype(np.float32).reshape(wl.B * wl.H, wl.nqb, wl.nkb)
+    rp, col, full = svg.adaspa_select(pb_of(wl), dev(m32), p)
+    svg.sync_status()
+    rp = rp.cpu().numpy()
+    n = int(rp[-1])
+    rp_r, col_r, full_r = oracle.adaspa_select(m32, wl.L, wl.Lv, wl.bq, wl.bk, p)
+    assert np.array_equal(rp, rp_r)
+    assert np.array_equal(col.cpu().numpy()[:n], col_r)
+    assert np.array_equal(full.cpu().numpy()[:n], full_r)
+
+
+@pytest.mark.parametrize("p", [0.3, 0.6, 0.99, 1.0])
+def test_select_bit_exact_random_masses_with_ties(p):
+    """Masses with exact ties and zeros, over several sort sizes."""
+    wl = W.small_workload(d=64, H=3, F=6, Hs=10, Ws=13, T=40, seed=2)   # nkb = 13
+    rng = np.random.Generator(np.random.PCG64(int(p * 100)))
+    m = rng.integers(0, 6, (wl.B * wl.H, wl.nqb, wl.nkb)).astype(np.float32) / 8
+    rp, col, full = svg.adaspa_select(pb_of(wl), dev(m), p)
+    svg.sync_status()
+    rp = rp.cpu().numpy()
+    rp_r, col_r, _ = oracle.adaspa_select(m, wl.L, wl.Lv, wl.bq, wl.bk, p)
+    assert np.array_equal(rp, rp_r)
+    assert np.array_equal(col.cpu().numpy()[:int(rp[-1])], col_r)
+
+
+def random_blocks(wl, keep=0.4, seed=3):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    k = rng.random((wl.B * wl.H * wl.nqb, wl.nkb)) < keep
+    k[:, 0] = True
+    rp = np.concatenate([[0], np.cumsum(k.sum(1))]).astype(np.int32)
+    col = np.concatenate([np.nonzero(r)[0] for r in k]).astype(np.int32)
+    return rp, col, np.ones(len(col), np.uint8)
+
+
+@pytest.mark.parametrize("key", list(CASES))
+def test_block_attention_parity(key):
+    """Attention over an arbitrary block list (every head DENSE, each listed
+    block computed whole) against the oracle's block attention."""
+    wl, p, inp, qn, kn, lse, tiles, _ = case(key)
+    rp, col, full = random_blocks(wl)
+    kinds = dev(np.full(wl.B * wl.H, W.DENSE, np.uint8))
+    out = svg.block_sparse_attn(pb_of(wl), dev(qn), dev(kn), dev(inp["v"]), kinds, dev(rp), dev(col), dev(full))
+    svg.sync_status()
+    rows = (np.arange(wl.B * wl.H * wl.L, dtype=np.int64) if key in SMALL
+            else W.random_rows(wl, 64, seed=17, boundary=False))
+    want = oracle.block_attention_rows(qn, kn, inp["v"], wl.bq, wl.bk, rp, col, rows)
+    assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], want, what=key)
+
+
+def clear_tiles(mass, wl, p, rel=1e-3):
+    """Query tiles whose top-p set is the same for every mass within `rel` of
+    the oracle's: no two video tiles near the cut within rel of each other,
+    and no running sum within rel of the goal."""
+    nv = wl.nkb if wl.L == wl.Lv else min(wl.nkb, wl.Lv // wl.bk)
+    ok = []
+    for m in mass.reshape(-1, wl.nkb):
+        v = np.sort(m[:nv])[::-1]
+        cum = np.cumsum(v)
+        goal = p * cum[-1]
+        cut = int(np.searchsorted(cum, goal * (1 - 1e-12)))
+        near = np.abs(cum - goal) < rel * cum[-1]
+        lo, hi = max(0, cut - 1), min(nv - 1, cut + 1)
+        gaps = np.abs(np.diff(v[lo:hi + 1])) < rel * v[lo:hi + 1].max(initial=0)
+        ok.append(not near.any() and not gaps.any())
+    return np.array(ok)
+
+
+def assert_valid_selection(kept, m, wl, qb, p, tol=1e-3):
+    """`kept` is a top-p set under masses m within tol: it holds the text tiles
+    (all tiles for a text query tile); its video tiles reach p of the video
+    mass, dropping the lightest falls below it, and no tile left out is
+    heavier than the lightest kept one."""
+    nv = wl.nkb if wl.L == wl.Lv else min(wl.nkb, wl.Lv // wl.bk)
+    if min(wl.L, (qb + 1) * wl.bq) > wl.Lv:
+        assert kept == list(range(wl.nkb))
+        return
+    assert [k for k in kept if k >= nv] == list(range(nv, wl.nkb))
+    kv = [k for k in kept if k < nv]
+    tot = m[:nv].sum()
+    mk = m[kv].sum()
+    assert mk >= p * tot - tol * tot
+    assert mk - m[kv].min() < p * tot + tol * tot
+    out = np.setdiff1d(np.arange(nv), kv)
+    if len(out):
+        assert m[out].max() <= m[kv].min() + tol * m[:nv].max()
+
+
+@pytest.mark.parametrize("key", list(CASES))
+def test_search_end_to_end(key):
+    """Masses and selection on the GPU.  Every query tile's kept set is a
+    valid top-p set under the oracle's masses within the mass tolerance, and
+    equals the oracle's own selection wherever that decision is clear of the
+    tolerance; the layer's sparse step matches the oracle's block attention."""
+    wl, p, inp, qn, kn, lse, tiles, mass = case(key)
+    layer = svg.AdaSpaLayer(pb_of(wl), p)
+    layer.lse = dev(lse)
+    layer.search(dev(qn), dev(kn))
+    out = layer.sparse(dev(qn), dev(kn), dev(inp["v"]))
+    svg.sync_status()
+    rp, col, _ = (t.cpu().numpy() for t in layer.blocks)
+    ids = np.arange(wl.B * wl.H * wl.nqb) if tiles is None else tiles
+    m_ref = mass.reshape(-1, wl.nkb)
+    for i, t in enumerate(ids):
+        assert_valid_selection(col[rp[t]:rp[t + 1]].tolist(), m_ref[i], wl, int(t) % wl.nqb, p)
+    clear = clear_tiles(m_ref, wl, p)
+    assert clear.sum() >= 1, f"{key}: no query tile is clear of the tolerance"
+    # the oracle's selection of the checked tiles, from its own masses
+    sub = m_ref.astype(np.float32).reshape(len(ids), 1, wl.nkb)
+    for i, t in enumerate(ids):
+        if not clear[i]:
+            continue
+        bh, qb = divmod(int(t), wl.nqb)
+        # one query tile at a time: a single-tile problem with the same L, Lv
+        one = np.zeros((1, wl.nqb, wl.nkb), np.float32)
+        one[0, qb] = sub[i, 0]
+        rp_r, col_r, _ = oracle.adaspa_select(one, wl.L, wl.Lv, wl.bq, wl.bk, p)
+        assert col[rp[t]:rp[t + 1]].tolist() == col_r[rp_r[qb]:rp_r[qb + 1]].tolist(), (key, int(t))
+    # attention rows of the clear tiles, over the GPU's (verified) lists
+    rows_local, which = rows_in_tiles(wl, ids[clear])
+    bhs = ids[clear] // wl.nqb
+    rows = bhs[which] * wl.L + rows_local
+    want = oracle.block_attention_rows(qn, kn, inp["v"], wl.bq, wl.bk, rp, col, rows)
+    assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], want, what=key)
+
+
+def test_layer_requires_lse_and_search():
+    wl, p, inp, qn, kn, lse, tiles, _ = case("d128")
+    layer = svg.AdaSpaLayer(pb_of(wl), p)
+    with pytest.raises(RuntimeError):
+        layer.search(dev(qn), dev(kn))
+    with pytest.raises(RuntimeError):
+        layer.sparse(dev(qn), dev(kn), dev(inp["v"]))
+    # a dense step caches the LSE; it matches the oracle's dense LSE
+    out = layer.dense(dev(qn), dev(kn), dev(inp["v"]))
+    svg.sync_status()
+    assert np.allclose(layer.lse.cpu().numpy(), lse, atol=2e-3)
+    assert out.shape == dev(qn).shape
+
+
+def test_bad_arguments_are_reported():
+    wl, p, inp, qn, kn, lse, tiles, mass = case("d128")
+    pb64 = svg.Problem.from_workload(wl, block_q=64)
+    with pytest.raises(RuntimeError):
+        svg.adaspa_block_mass(pb64, dev(qn), dev(kn), dev(lse),
+                              out=torch.empty(wl.B * wl.H * pb64.nqb * pb64.nkb, device="cuda"))
+    with pytest.raises(RuntimeError):
+        svg.adaspa_select(pb_of(wl), dev(mass.astype(np.float32)), 0.0)
+    svg.sync_status()

@@ -151,3 +151,12 @@ def test_search_then_attention_keeps_at_least_p_of_each_tiles_mass():
         # and it is the shortest such set: dropping the lightest kept tile falls below p
         if len(kept) > 1:
             assert mt[kept].sum() - mt[kept].min() < p * mt.sum()
+
+
+def test_mass_of_chosen_tiles_equals_the_full_computation():
+    q, k, _ = _qkv(L=50, d=16, seed=13)
+    lse = _dense_lse(q, k)
+    full = oracle.block_mass(q, k, lse, 16, 8)
+    tiles = np.array([5, 0, 3], np.int64)                 # bh * nqb + qb, nqb = 4
+    part = oracle.block_mass(q, k, lse, 16, 8, tiles=tiles)
+    assert np.array_equal(part, full.reshape(-1, full.shape[2])[tiles])
