@@ -315,12 +315,15 @@ __device__ __forceinline__ long long sel_block_scan(long long v, long long* warp
   return v + base;
 }
 
-// FILL = false: row_ptr[t + 1] = number of kept tiles; FILL = true: the kept
-// tiles in increasing order at col[row_ptr[t] ...], full = 1.
+// FILL = false: row_ptr[t + 1] = number of kept tiles, and with `stash` the
+// kept flags at stash[t * nkb + kb]; FILL = true: the kept tiles in increasing
+// order at col[row_ptr[t] ...] and full = 1, or with `stash` the flags read
+// back from it (no second sort) and col alone written (stash aliases full,
+// which the caller then sets to 1).
 template <bool FILL>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a, int32_t* __restrict__ row_ptr,
-                                                            int32_t* __restrict__ col, uint8_t* __restrict__ full,
-                                                            int64_t capacity, int P2) {
+                                                            int32_t* __restrict__ col, uint8_t* full,
+                                                            int64_t capacity, int P2, uint8_t* stash) {
   extern __shared__ uint8_t sel_smem[];
   float* sm = reinterpret_cast<float*>(sel_smem);              // [P2] masses, sorted in place
   int* si = reinterpret_cast<int*>(sm + P2);                    // [P2] tile indices
@@ -335,17 +338,27 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a, in
   const bool text_q = min(g.L, (qb + 1) * g.bq) > g.Lv;
   // video key tiles: no key in [Lv, L) (without text, every tile)
   const int nv = (g.L == g.Lv) ? g.nkb : min(g.nkb, g.Lv / g.bk);
+  const bool reuse = FILL && stash;
   for (int i = tid; i < P2; i += kSelThreads) {
     const bool vid = i < nv;
+    if (reuse) {
+      keep[i] = (i < g.nkb) ? stash[t * g.nkb + i] : 0;
+      continue;
+    }
     sm[i] = vid ? __ldg(m + i) : -INFINITY;
     si[i] = i;
     keep[i] = (i < g.nkb && (text_q || !vid)) ? 1 : 0;
   }
   __syncthreads();
-  if (!text_q && nv > 0) {
-    // bitonic sort of (mass, index): heavier first, the lower index first on ties
-    for (int k = 2; k <= P2; k <<= 1)
-      for (int jj = k >> 1; jj > 0; jj >>= 1) {
+  if (!reuse && !text_q && nv > 0) {
+    // bitonic sort of (mass, index): heavier first, the lower index first on ties.
+    // Exchanges 64 or more positions apart go through shared memory; the rest run
+    // in registers inside 64-position segments (lane and lane + 32 of a warp),
+    // by shuffles.
+    const int lane = tid & 31, warp = tid >> 5;
+    for (int k = 2; k <= P2; k <<= 1) {
+      int jj = k >> 1;
+      for (; jj >= 64; jj >>= 1) {
         for (int i = tid; i < P2; i += kSelThreads) {
           const int l = i ^ jj;
           if (l > i) {
@@ -363,6 +376,45 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a, in
         }
         __syncthreads();
       }
+      for (int seg = warp; seg < P2 / 64; seg += kSelThreads / 32) {
+        const int pa = seg * 64 + lane, pb = pa + 32;
+        float ma = sm[pa], mb = sm[pb];
+        int ia = si[pa], ib = si[pb];
+        if (jj == 32) {                                 // partners in the same thread
+          const bool up = (pa & k) == 0;
+          if (up ? sel_before(mb, ib, ma, ia) : sel_before(ma, ia, mb, ib)) {
+            const float tm = ma;
+            const int ti = ia;
+            ma = mb;
+            ia = ib;
+            mb = tm;
+            ib = ti;
+          }
+        }
+        for (int j = min(jj, 16); j > 0; j >>= 1) {
+#pragma unroll
+          for (int e = 0; e < 2; e++) {
+            float& m = e ? mb : ma;
+            int& ix = e ? ib : ia;
+            const int pos = e ? pb : pa;
+            const float om = __shfl_xor_sync(0xffffffffu, m, j);
+            const int oi = __shfl_xor_sync(0xffffffffu, ix, j);
+            // the lower position of the pair takes the element that comes first in
+            // an ascending run, the other one in a descending run
+            const bool want_first = ((pos & j) == 0) == ((pos & k) == 0);
+            if (want_first != sel_before(m, ix, om, oi)) {
+              m = om;
+              ix = oi;
+            }
+          }
+        }
+        sm[pa] = ma;
+        sm[pb] = mb;
+        si[pa] = ia;
+        si[pb] = ib;
+      }
+      __syncthreads();
+    }
     // fixed-point masses in sorted order: each thread owns P2 / kSelThreads consecutive positions
     const int per = P2 / kSelThreads > 0 ? P2 / kSelThreads : 1;
     const int p0 = tid * per;
@@ -402,6 +454,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a, in
   if (!FILL) {
     if (tid == kSelThreads - 1) row_ptr[t + 1] = static_cast<int32_t>(incl);
     if (t == 0 && tid == 0) row_ptr[0] = 0;
+    if (stash)
+      for (int i = tid; i < g.nkb; i += kSelThreads) stash[t * g.nkb + i] = keep[i];
     return;
   }
   int64_t e = row_ptr[t] + (incl - cnt);
@@ -410,7 +464,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelArgs a, in
     if (kb < g.nkb && keep[kb]) {
       if (e < capacity) {
         col[e] = kb;
-        full[e] = 1;
+        if (!stash) full[e] = 1;
       }
       e++;
     }

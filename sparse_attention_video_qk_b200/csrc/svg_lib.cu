@@ -797,17 +797,24 @@ svg_status svg_adaspa_select(const svg_shape* s, const svg_params* p, const floa
   a.p = top_p;
   a.mass = mass;
   if (a.g.nkb > kSelMaxTiles) return SVG_ERR_UNSUPPORTED;
-  int P2 = 2;
+  int P2 = 64;                                   // the sort works on 64-position segments
   while (P2 < a.g.nkb) P2 <<= 1;
   const int smem = P2 * 9;
   const int64_t n = static_cast<int64_t>(a.g.BH) * a.g.nqb;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  select_kernel<false><<<static_cast<unsigned>(n), kSelThreads, smem, cs>>>(a, row_ptr, col, full, capacity, P2);
+  // with room for every tile's flags, `full` keeps them between the passes (no second sort)
+  const bool room = capacity >= n * a.g.nkb;
+  uint8_t* stash = room ? full : nullptr;
+  select_kernel<false><<<static_cast<unsigned>(n), kSelThreads, smem, cs>>>(a, row_ptr, col, full, capacity, P2,
+                                                                            stash);
   if ((st = launch_status()) != SVG_OK) return st;
   block_scan_kernel<<<1, 1024, 0, cs>>>(row_ptr, n, capacity);
   if ((st = launch_status()) != SVG_OK) return st;
-  select_kernel<true><<<static_cast<unsigned>(n), kSelThreads, smem, cs>>>(a, row_ptr, col, full, capacity, P2);
-  return launch_status();
+  select_kernel<true><<<static_cast<unsigned>(n), kSelThreads, smem, cs>>>(a, row_ptr, col, full, capacity, P2,
+                                                                           stash);
+  if ((st = launch_status()) != SVG_OK) return st;
+  if (room && cudaMemsetAsync(full, 1, static_cast<size_t>(capacity), cs) != cudaSuccess) return SVG_ERR_CUDA;
+  return SVG_OK;
 }
 
 }  // extern "C"

@@ -120,6 +120,20 @@ def test_select_bit_exact_on_the_same_masses(key):
     assert np.array_equal(full.cpu().numpy()[:n], full_r)
 
 
+def test_select_with_a_tight_capacity_matches():
+    """Capacity below one flag per tile: the fill pass sorts again instead of
+    reading the flags back; the lists are the same."""
+    wl, p, inp, qn, kn, lse, tiles, mass = case("d128")
+    m32 = dev(mass.astype(np.float32).reshape(wl.B * wl.H, wl.nqb, wl.nkb))
+    rp, col, full = svg.adaspa_select(pb_of(wl), m32, p)
+    n = int(rp[-1])
+    rp2, col2, full2 = svg.adaspa_select(pb_of(wl), m32, p, capacity=n)
+    svg.sync_status()
+    assert n < wl.B * wl.H * wl.nqb * wl.nkb
+    assert torch.equal(rp, rp2)
+    assert torch.equal(col[:n], col2[:n]) and torch.equal(full[:n], full2[:n])
+
+
 @pytest.mark.parametrize("p", [0.3, 0.6, 0.99, 1.0])
 def test_select_bit_exact_random_masses_with_ties(p):
     """Masses with exact ties and zeros, over several sort sizes."""
