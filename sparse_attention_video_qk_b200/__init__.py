@@ -19,6 +19,17 @@ quarter of the steps, then profiled), and ``sparse_attention`` /
 ``HostPipeline`` take pinned host tensors and overlap the copies with the
 computation.  Each stage is also callable on its own (``qknorm_rope_layout``,
 ``profile_heads``, ``build_block_index``, ``block_sparse_attn``, ...).
+
+Two further sparse-attention methods run on the same kernels, on normalised
+Q and K (``qknorm_rope``)::
+
+    svg2 = svg.SVG2Layer(pb, Cq=64, Ck=64, iters=2, top_p=0.9)   # semantic-aware permutation
+    out = svg2(qn, kn, v)            # k-means (warm-started on later calls), sort, top-p, attention
+
+    ada = svg.AdaSpaLayer(pb, top_p=0.9)                       # blockified LSE-cached search
+    out = ada.dense(qn, kn, v)       # a dense step keeps every row's LSE
+    ada.search(qn, kn)               # block masses under that LSE -> kept tiles
+    out = ada.sparse(qn, kn, v)      # later steps reuse the pattern
 """
 from ._lib import SVGError, lib  # noqa: F401
 from .api import (DENSE, SPATIAL, TEMPORAL, Problem, StepBuffers, attention_step,  # noqa: F401

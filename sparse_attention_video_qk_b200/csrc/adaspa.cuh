@@ -6,13 +6,13 @@
 // 1. mass_kernel: the exact attention mass of every (query tile, key tile)
 //    block, given each row's log-sum-exp from an earlier step:
 //        M[qb][kb] = sum_{q in qb, k in kb} 2^(s_qk * scale * log2 e - lse_q * log2 e)
-//    in one pass over Q K^T (no normalisation pass: the LSE is known).  The
-//    CTA layout follows the attention kernel: one CTA per (b, h, pair of
-//    128-row query tiles), warp 0 streams K through a TMA slot ring, warp 1
-//    issues S = Q K^T as M=128, N=128 tcgen05 MMAs into TMEM, warps 2-5 and
-//    6-9 exponentiate and sum the two query tiles' S (thread = row).  S is
-//    double-buffered per query tile (4 x 128 TMEM columns), so the MMAs of
-//    tile j+1 overlap the exponentials of tile j.  The per-row sums of each
+//    in one pass over Q K^T (no normalisation pass: the LSE is known).  One
+//    CTA per (b, h, set of NG 128-row query tiles): warp 0 streams K through a
+//    TMA slot ring, warp 1 issues S = Q K^T as M=128, N=128 tcgen05 MMAs into
+//    TMEM, and each following group of 4 warps exponentiates and sums one query
+//    tile's S (thread = row).  With NG = 4 (the default) each group's S is one
+//    128-column TMEM buffer and the other groups' MMAs run while a group
+//    exponentiates; with NG = 2 it is double-buffered.  The per-row sums of each
 //    64-key block are reduced over the tile's 128 rows by shuffles and a fixed
 //    4-warp order, so the result does not depend on scheduling.
 // 2. select_kernel: per (head, query tile), the video key tiles sorted by
@@ -31,23 +31,43 @@
 
 namespace svg {
 
-template <int D>
+// NG query tiles per CTA (one softmax group of 4 warps each).  With NG = 2 each
+// group's S is double-buffered in TMEM; with NG = 4 single-buffered, and the
+// other groups' MMAs fill the tensor pipe while one group exponentiates.
+template <int D, int NG>
 struct MassCfg {
   static constexpr int PANELS = D / 64;
   static constexpr int PANEL = 128 * 128;          // bytes of one 128-row panel
   static constexpr int Q_BYTES = 128 * D * 2;      // one query tile
   static constexpr int SLOT_BYTES = 128 * D * 2;   // one 128-key K tile
-  static constexpr int NSLOT = (D == 128) ? 4 : 8;
-  static constexpr int DATA_BYTES = 2 * Q_BYTES + NSLOT * SLOT_BYTES;
-  static constexpr int BAR_BYTES = 512;
+  static constexpr int NBUF = (NG == 2) ? 2 : 1;   // S buffers per group
+  static constexpr int NSLOT = (NG == 2) ? ((D == 128) ? 4 : 8) : ((D == 128) ? 3 : 8);
+  static constexpr int DATA_BYTES = NG * Q_BYTES + NSLOT * SLOT_BYTES;
+  static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM_BYTES = DATA_BYTES + BAR_BYTES + 1024;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 64 + 128 * NG;
   static constexpr uint32_t TMEM_COLS = 512;
-  // TMEM columns: S of query tile w, buffer b at 256*w + 128*b
-  static __device__ __forceinline__ uint32_t tm_s(int w, int b) { return 256u * w + 128u * b; }
+  static __device__ __forceinline__ uint32_t tm_s(int w, int b) { return 128u * (NBUF * w + b); }
+  // barrier slots (8 bytes each): q, full[NSLOT], empty[NSLOT], s[NG][NBUF], free[NG][NBUF],
+  // part[NG][2], pfree[NG][2], drain, the TMEM slot, the abort flag, then the partial sums
+  static constexpr int BAR_S = 1 + 2 * NSLOT;
+  static constexpr int BAR_FREE = BAR_S + NG * NBUF;
+  static constexpr int BAR_PART = BAR_FREE + NG * NBUF;
+  static constexpr int BAR_PFREE = BAR_PART + 2 * NG;
+  static constexpr int BAR_DRAIN = BAR_PFREE + 2 * NG;
+  static constexpr int SLOT_TMEM = BAR_DRAIN + 1;
+  static constexpr int SLOT_ABORT = SLOT_TMEM + 1;
+  static constexpr int SLOT_PART = SLOT_ABORT + 1;  // NG * 2 bufs * 4 warps * 2 floats
+  static_assert(NBUF * NG * 128 <= 512, "TMEM columns");
+  static_assert(SLOT_PART + NG * 8 <= BAR_BYTES / 8, "barrier area");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(20 + 2 * NSLOT + 16 <= BAR_BYTES / 8, "barrier area");
 };
+
+// query tiles per CTA of the block-mass launch
+#ifndef SVG_MASS_GROUPS
+#define SVG_MASS_GROUPS 4
+#endif
+constexpr int kMassGroups = SVG_MASS_GROUPS;
 
 struct MassArgs {
   Geometry g;
@@ -56,35 +76,33 @@ struct MassArgs {
   float* mass;             // [BH][nqb][nkb]
 };
 
-template <int D>
-__global__ void __launch_bounds__(MassCfg<D>::THREADS, 1)
+template <int D, int NG>
+__global__ void __launch_bounds__(MassCfg<D, NG>::THREADS, 1)
     mass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const MassArgs a) {
-  using C = MassCfg<D>;
-  constexpr int NSLOT = C::NSLOT;
+  using C = MassCfg<D, NG>;
+  constexpr int NSLOT = C::NSLOT, NBUF = C::NBUF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + 2 * C::Q_BYTES;
+  uint8_t* sK = smem + NG * C::Q_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::DATA_BYTES);
-  // barriers: q | full[NSLOT] | empty[NSLOT] | s[2][2] | free[2][2] | part[2][2] | pfree[2][2] |
-  // drain; then the TMEM slot, the abort flag and the per-warp partial sums
   const uint32_t b_q = smem_addr(&bars[0]);
   auto b_full = [&](int s) { return smem_addr(&bars[1 + s]); };
   auto b_empty = [&](int s) { return smem_addr(&bars[1 + NSLOT + s]); };
-  auto b_s = [&](int w, int b) { return smem_addr(&bars[1 + 2 * NSLOT + 2 * w + b]); };
-  auto b_free = [&](int w, int b) { return smem_addr(&bars[5 + 2 * NSLOT + 2 * w + b]); };
-  auto b_part = [&](int w, int b) { return smem_addr(&bars[9 + 2 * NSLOT + 2 * w + b]); };
-  auto b_pfree = [&](int w, int b) { return smem_addr(&bars[13 + 2 * NSLOT + 2 * w + b]); };
-  const uint32_t b_drain = smem_addr(&bars[17 + 2 * NSLOT]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[18 + 2 * NSLOT]);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[19 + 2 * NSLOT]);
-  float* part = reinterpret_cast<float*>(&bars[20 + 2 * NSLOT]);   // [2 groups][2 bufs][4 warps][2]
+  auto b_s = [&](int w, int b) { return smem_addr(&bars[C::BAR_S + NBUF * w + b]); };
+  auto b_free = [&](int w, int b) { return smem_addr(&bars[C::BAR_FREE + NBUF * w + b]); };
+  auto b_part = [&](int w, int b) { return smem_addr(&bars[C::BAR_PART + 2 * w + b]); };
+  auto b_pfree = [&](int w, int b) { return smem_addr(&bars[C::BAR_PFREE + 2 * w + b]); };
+  const uint32_t b_drain = smem_addr(&bars[C::BAR_DRAIN]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[C::SLOT_TMEM]);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&bars[C::SLOT_ABORT]);
+  float* part = reinterpret_cast<float*>(&bars[C::SLOT_PART]);   // [NG groups][2 bufs][4 warps][2]
 
   const Geometry& g = a.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int npair = (g.nqb + 1) >> 1;
-  const int bh = blockIdx.x / npair, qb0 = 2 * (blockIdx.x % npair);
+  const int nset = (g.nqb + NG - 1) / NG;             // sets of NG query tiles per head
+  const int bh = blockIdx.x / nset, qb0 = NG * (blockIdx.x % nset);
   const int ntile = (g.nkb + 1) >> 1;                  // 128-key tiles: blocks 2j, 2j+1
 
   if (threadIdx.x == 0) {
@@ -93,13 +111,16 @@ __global__ void __launch_bounds__(MassCfg<D>::THREADS, 1)
       mbar_init(b_full(s), 1);
       mbar_init(b_empty(s), 1);
     }
-    for (int w = 0; w < 2; w++)
-      for (int b = 0; b < 2; b++) {
+    for (int w = 0; w < NG; w++) {
+      for (int b = 0; b < NBUF; b++) {
         mbar_init(b_s(w, b), 1);
         mbar_init(b_free(w, b), 128);
+      }
+      for (int b = 0; b < 2; b++) {
         mbar_init(b_part(w, b), 4);
         mbar_init(b_pfree(w, b), 1);
       }
+    }
     mbar_init(b_drain, 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -115,9 +136,9 @@ __global__ void __launch_bounds__(MassCfg<D>::THREADS, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmq);
       tma_prefetch_desc(&tmk);
-      mbar_expect_tx(b_q, 2 * C::Q_BYTES);
+      mbar_expect_tx(b_q, NG * C::Q_BYTES);
 #pragma unroll
-      for (int w = 0; w < 2; w++)
+      for (int w = 0; w < NG; w++)
 #pragma unroll
         for (int p = 0; p < C::PANELS; p++)
           tma_load_3d(smem_addr(sQ + w * C::Q_BYTES + p * C::PANEL), &tmq, p * 64, (qb0 + w) * 128, bh, b_q);
@@ -148,12 +169,12 @@ __global__ void __launch_bounds__(MassCfg<D>::THREADS, 1)
       bool issued_any = false;
       bool ok = mbar_wait(b_q, 0, abort_flag);
       for (int j = 0; ok && j < ntile; j++) {
-        const int st = j % NSLOT, b = j & 1;
+        const int st = j % NSLOT, b = j % NBUF;
         const int nb = (2 * j + 1 < g.nkb) ? 2 : 1;
         if (!mbar_wait(b_full(st), (j / NSLOT) & 1, abort_flag)) break;
-        for (int w = 0; w < 2 && ok; w++) {
-          // S_w buffer b was last read by the softmax at tile j-2
-          if (j >= 2 && !mbar_wait(b_free(w, b), ((j >> 1) - 1) & 1, abort_flag)) {
+        for (int w = 0; w < NG && ok; w++) {
+          // S_w buffer b was last read by the softmax at tile j - NBUF
+          if (j >= NBUF && !mbar_wait(b_free(w, b), ((j / NBUF) - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -176,7 +197,7 @@ __global__ void __launch_bounds__(MassCfg<D>::THREADS, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ exponentials (two groups)
+    // ------------------------------------------------------------ exponentials (NG groups)
     const int w = (warp - 2) >> 2;                 // query tile of this group
     const int q4 = warp & 3;                       // TMEM lane quarter
     const int wg = (warp - 2) & 3;                 // warp index inside the group
@@ -191,8 +212,8 @@ __global__ void __launch_bounds__(MassCfg<D>::THREADS, 1)
     const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     float* mrow = a.mass + (static_cast<int64_t>(bh) * g.nqb + qb0 + w) * g.nkb;
     for (int j = 0; j < ntile; j++) {
-      const int b = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(b_s(w, b), (j >> 1) & 1, abort_flag))) break;
+      const int b = j % NBUF;
+      if (!__all_sync(0xffffffffu, mbar_wait(b_s(w, b), (j / NBUF) & 1, abort_flag))) break;
       tc_fence_after();
       const uint32_t tS = tl + C::tm_s(w, b);
       float h[2];
@@ -238,25 +259,26 @@ __global__ void __launch_bounds__(MassCfg<D>::THREADS, 1)
         h[0] += __shfl_xor_sync(0xffffffffu, h[0], o);
         h[1] += __shfl_xor_sync(0xffffffffu, h[1], o);
       }
-      float* pb = part + ((w * 2 + b) * 4) * 2;
+      const int hb = j & 1;                        // hand-off buffer
+      float* pb = part + ((w * 2 + hb) * 4) * 2;
       int okp = 1;
       if (lane == 0) {
-        if (j >= 2) okp = mbar_wait(b_pfree(w, b), ((j >> 1) - 1) & 1, abort_flag);
+        if (j >= 2) okp = mbar_wait(b_pfree(w, hb), ((j >> 1) - 1) & 1, abort_flag);
         if (okp) {
           pb[wg * 2] = h[0];
           pb[wg * 2 + 1] = h[1];
-          mbar_arrive(b_part(w, b));
+          mbar_arrive(b_part(w, hb));
         }
       }
       if (!__shfl_sync(0xffffffffu, okp, 0)) break;
       if (wg == 0) {
         int okr = 1;
         if (lane == 0) {
-          okr = mbar_wait(b_part(w, b), (j >> 1) & 1, abort_flag);
+          okr = mbar_wait(b_part(w, hb), (j >> 1) & 1, abort_flag);
           if (okr) {
             const float m0 = ((pb[0] + pb[2]) + pb[4]) + pb[6];
             const float m1 = ((pb[1] + pb[3]) + pb[5]) + pb[7];
-            mbar_arrive(b_pfree(w, b));
+            mbar_arrive(b_pfree(w, hb));
             if (tile_ok) {
               mrow[2 * j] = m0;
               if (2 * j + 1 < g.nkb) mrow[2 * j + 1] = m1;

@@ -775,14 +775,16 @@ svg_status svg_adaspa_block_mass(const svg_shape* s, const svg_params* p, const 
   a.mass = mass;
   CUtensorMap mq, mk;
   if (!make_map(&mq, q, s->d, s->L, a.g.BH, 128) || !make_map(&mk, k, s->d, s->L, a.g.BH, 64)) return SVG_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(a.g.BH) * static_cast<unsigned>((a.g.nqb + 1) / 2);
+  constexpr int NG = kMassGroups;
+  const unsigned grid = static_cast<unsigned>(a.g.BH) * static_cast<unsigned>((a.g.nqb + NG - 1) / NG);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  auto run = [&](auto kern, int smem) -> svg_status {
+  auto run = [&](auto kern, int threads, int smem) -> svg_status {
     if (!set_smem(kern, smem)) return SVG_ERR_CUDA;
-    kern<<<grid, MassCfg<128>::THREADS, smem, cs>>>(mq, mk, a);
+    kern<<<grid, threads, smem, cs>>>(mq, mk, a);
     return launch_status();
   };
-  return s->d == 128 ? run(mass_kernel<128>, MassCfg<128>::SMEM_BYTES) : run(mass_kernel<64>, MassCfg<64>::SMEM_BYTES);
+  if (s->d == 128) return run(mass_kernel<128, NG>, MassCfg<128, NG>::THREADS, MassCfg<128, NG>::SMEM_BYTES);
+  return run(mass_kernel<64, NG>, MassCfg<64, NG>::THREADS, MassCfg<64, NG>::SMEM_BYTES);
 }
 
 svg_status svg_adaspa_select(const svg_shape* s, const svg_params* p, const float* mass, double top_p,

@@ -271,3 +271,29 @@ def test_bad_arguments_are_reported():
     with pytest.raises(RuntimeError):
         svg.adaspa_select(pb_of(wl), dev(mass.astype(np.float32)), 0.0)
     svg.sync_status()
+
+
+def test_select_capacity_overflow_is_reported():
+    """A capacity below the kept count: the scan records SVG_ERR_CAPACITY and
+    nothing is written past the capacity."""
+    wl, p, inp, qn, kn, lse, tiles, mass = case("d128")
+    m32 = dev(mass.astype(np.float32).reshape(wl.B * wl.H, wl.nqb, wl.nkb))
+    rp, col, full = svg.adaspa_select(pb_of(wl), m32, p)
+    n = int(rp[-1])
+    svg.sync_status()
+    cap = n // 2
+    col2 = torch.full((n,), -7, dtype=torch.int32, device="cuda")
+    full2 = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    rp2 = torch.empty_like(rp)
+    from sparse_attention_video_qk_b200._lib import check
+    import ctypes
+    pb = pb_of(wl)
+    sh, pr = pb.c_shape(), pb.c_params()
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    check(svg.lib().svg_adaspa_select(ctypes.byref(sh), ctypes.byref(pr), P(m32), float(p), P(rp2), P(col2),
+                                      P(full2), cap, None), "svg_adaspa_select")
+    with pytest.raises(svg.SVGError) as e:
+        svg.sync_status()
+    assert e.value.status == 5
+    assert (col2[cap:].cpu().numpy() == -7).all()
+    svg.sync_status()

@@ -327,3 +327,18 @@ def test_bad_arguments_are_reported():
     with pytest.raises(RuntimeError):
         svg.svg2_attention(pb64, dev(qn), dev(kn), dev(inp["v"]), qoff, koff, sel, dev(ref["pq"]), rp, col, full)
     svg.sync_status()
+
+
+def test_block_index_capacity_overflow_is_reported():
+    wl, inp, qn, kn, ref = case("d128")
+    pb = pb_of(wl)
+    qoff, koff, sel = dev(ref["qoff"]), dev(ref["koff"]), dev(ref["sel"].view(np.int64))
+    rp, col, full = svg.svg2_block_index(pb, qoff, koff, sel)
+    n = int(rp[-1])
+    svg.sync_status()
+    cap = n // 2
+    rp2, col2, full2 = svg.svg2_block_index(pb, qoff, koff, sel, capacity=cap)
+    with pytest.raises(svg.SVGError) as e:
+        svg.sync_status()
+    assert e.value.status == 5
+    svg.sync_status()
