@@ -57,16 +57,10 @@ __global__ void km_init_kernel(const KmArgs a) {
 // load gives two dimensions of two centroids and one packed FMA advances two
 // dot products; a pass covers kKmGroup pairs (8 centroids) with one unpacking
 // of each x_i.
-constexpr int kKmGroup = 4;                              // centroid pairs per pass (padding unit)
+constexpr int kKmGroup = 4;                              // centroid pairs per pass
 
 __host__ __device__ constexpr int km_assign_pairs(int C) {
   return (C + 2 * kKmGroup - 1) / (2 * kKmGroup) * kKmGroup;   // padded to whole passes
-}
-
-// pairs per pass: fewer at d = 128, where the two rows take 128 registers
-template <int D>
-__host__ __device__ constexpr int km_group() {
-  return D == 128 ? 4 : 4;
 }
 
 // shared memory of km_assign_kernel: the pairs, then |c|^2 of every (padded) centroid
@@ -139,7 +133,7 @@ __global__ void __launch_bounds__(kKmAssignThreads, 1) km_assign_kernel(const Km
     km_load_row<D>(a, bh, r1, xw1);
     int best0 = 0, best1 = 0;
     float bestd0 = INFINITY, bestd1 = INFINITY;
-    constexpr int G = km_group<D>();
+    constexpr int G = kKmGroup;
     for (int g = 0; g < npair; g += G) {
       uint64_t acc0[G], acc1[G];
 #pragma unroll
