@@ -46,14 +46,16 @@ def dense_lse(qn, kn, wl, tiles=None):
     the LSE a dense step would cache.  With `tiles`, only the rows of those
     query tiles; the other rows get log(L)."""
     BH, L, d = wl.B * wl.H, wl.L, wl.d
-    q = W.bf16_bits_to_f32(qn.reshape(BH, L, d)).astype(np.float64)
-    k = W.bf16_bits_to_f32(kn.reshape(BH, L, d)).astype(np.float64)
+    qh, kh = qn.reshape(BH, L, d), kn.reshape(BH, L, d)
     lse = np.full((BH, L), np.log(L), np.float64)
     todo = range(BH * wl.nqb) if tiles is None else tiles
+    kf = {}
     for t in todo:
         bh, qb = divmod(int(t), wl.nqb)
+        if bh not in kf:
+            kf = {bh: W.bf16_bits_to_f32(kh[bh]).astype(np.float64)}     # one head's keys at a time
         r0, r1 = qb * wl.bq, min(L, (qb + 1) * wl.bq)
-        s = q[bh, r0:r1] @ k[bh].T / np.sqrt(d)
+        s = W.bf16_bits_to_f32(qh[bh, r0:r1]).astype(np.float64) @ kf[bh].T / np.sqrt(d)
         m = s.max(1, keepdims=True)
         lse[bh, r0:r1] = m[:, 0] + np.log(np.exp(s - m).sum(1))
     return lse.astype(np.float32).reshape(wl.B, wl.H, L)
@@ -297,3 +299,34 @@ def test_select_capacity_overflow_is_reported():
     assert e.value.status == 5
     assert (col2[cap:].cpu().numpy() == -7).all()
     svg.sync_status()
+
+
+def test_search_at_the_hunyuanvideo_shape_on_sampled_tiles():
+    """Block masses, selection and the sparse step at the HunyuanVideo 720p
+    shape (24 heads, 931 query tiles x 1861 key tiles per head) on sampled
+    query tiles, with the oracle's LSE for their rows."""
+    wl, p = W.HUNYUAN, 0.9
+    inp = W.make_inputs(wl)
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    qn = oracle.qknorm_rope(sh, pr, inp["q"], inp["gamma_q"])
+    kn = oracle.qknorm_rope(sh, pr, inp["k"], inp["gamma_k"])
+    rng = np.random.Generator(np.random.PCG64(9))
+    tiles = np.sort(rng.choice(wl.B * wl.H * wl.nqb, 6, replace=False)).astype(np.int64)
+    tiles = np.unique(np.concatenate([tiles, [wl.nqb - 1, 2 * wl.nqb - 2]])).astype(np.int64)
+    lse = dense_lse(qn, kn, wl, tiles)
+    want = oracle.block_mass(qn, kn, lse, wl.bq, wl.bk, tiles=tiles)
+    layer = svg.AdaSpaLayer(pb_of(wl), p)
+    layer.lse = dev(lse)
+    mass = layer.search(dev(qn), dev(kn))
+    out = layer.sparse(dev(qn), dev(kn), dev(inp["v"]))
+    svg.sync_status()
+    got = mass.cpu().numpy().reshape(-1, wl.nkb)[tiles].astype(np.float64)
+    assert (np.abs(got - want) <= 2e-4 * want + 1e-6 * wl.bq).all()
+    rp, col, _ = (t.cpu().numpy() for t in layer.blocks)
+    for i, t in enumerate(tiles):
+        assert_valid_selection(col[rp[t]:rp[t + 1]].tolist(), want[i], wl, int(t) % wl.nqb, p)
+    rows_local, which = rows_in_tiles(wl, tiles[:3])
+    rows_local, which = rows_local[::8], which[::8]               # every 8th row of three tiles
+    rows = (tiles[:3] // wl.nqb)[which] * wl.L + rows_local
+    ref = oracle.block_attention_rows(qn, kn, inp["v"], wl.bq, wl.bk, rp, col, rows)
+    assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, what="hunyuan")

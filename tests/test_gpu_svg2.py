@@ -342,3 +342,37 @@ def test_block_index_capacity_overflow_is_reported():
         svg.sync_status()
     assert e.value.status == 5
     svg.sync_status()
+
+
+def test_layer_at_the_hunyuanvideo_shape_on_two_heads():
+    """The whole layer at the HunyuanVideo 720p shape (24 heads, 119,056
+    tokens, 64 + 64 clusters), checked on one planted-spatial and one
+    planted-temporal head: centroids, sort and top-p bit-exact, attention on
+    sampled rows (every step is per head, so two heads of the oracle stand
+    for the launch)."""
+    wl = W.HUNYUAN
+    inp = W.make_inputs(wl)
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    qn = oracle.qknorm_rope(sh, pr, inp["q"], inp["gamma_q"])
+    kn = oracle.qknorm_rope(sh, pr, inp["k"], inp["gamma_k"])
+    layer = svg.SVG2Layer(pb_of(wl), 64, 64, 2, 0.9)
+    out = layer(dev(qn), dev(kn), dev(inp["v"]))
+    svg.sync_status()
+    heads = [0, 1]
+    q2, k2, v2 = (np.ascontiguousarray(x[:, heads]) for x in (qn, kn, inp["v"]))
+    cq, aq, nq = oracle.kmeans(q2, wl.Lv, 64, 2)
+    ck, ak, nk = oracle.kmeans(k2, wl.Lv, 64, 2)
+    pq, qoff = oracle.cluster_permutation(aq, 64)
+    sel, weight = oracle.select_top_p(cq, ck, nk, 1.0 / np.sqrt(wl.d), 0.9, want_weight=True)
+    assert clear_decisions(weight, 0.9).all()
+    assert np.array_equal(f32_bits(host(layer.cq)[heads]), f32_bits(cq))
+    assert np.array_equal(f32_bits(host(layer.ck)[heads]), f32_bits(ck))
+    assert np.array_equal(host(layer.last["perm_q"])[heads], pq)
+    assert np.array_equal(host(layer.last["qoff"])[heads], qoff)
+    assert np.array_equal(host(layer.last["sel"]).view(np.uint64)[heads], sel)
+    rng = np.random.Generator(np.random.PCG64(3))
+    toks = np.unique(np.concatenate([rng.choice(wl.L, 40, replace=False), np.arange(wl.L - 8, wl.L)]))
+    rows = np.concatenate([h * wl.L + toks for h in range(2)]).astype(np.int64)
+    want = oracle.attention2_rows(q2, k2, v2, wl.Lv, aq, ak, sel, rows)
+    got = host_bits(out).reshape(wl.H, wl.L, wl.d)[heads].reshape(-1, wl.d)[rows]
+    assert_attention_close(got, want, what="hunyuan")
