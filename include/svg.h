@@ -277,7 +277,8 @@ svg_status svg2_kmeans(const svg_shape* shape, const uint16_t* x, int C, int ite
 
 /* Stable counting sort of each head's video rows by cluster: perm (device int32
  * [B*H][Lv]) = the row placed at each position, off (device int32 [B*H][C+1]) =
- * the first position of each cluster (off[C] = Lv). */
+ * the first position of each cluster (off[C] = Lv).  An assignment outside
+ * [0, C) is left out and reported as SVG_ERR_INVALID_ARG by svg_sync_status. */
 svg_status svg2_permutation(const svg_shape* shape, const uint8_t* assign, int C, int32_t* perm, int32_t* off,
                             void* stream);
 
@@ -293,7 +294,9 @@ svg_status svg2_select(const svg_shape* shape, const svg_params* params, const f
                        const int32_t* counts_k, int Cq, int Ck, double top_p, uint64_t* sel, void* stream);
 
 /* Q, K, V into cluster order: video position p of q_out takes row perm_q[p];
- * k_out and v_out take row perm_k[p]; text rows are copied in place. */
+ * k_out and v_out take row perm_k[p]; text rows are copied in place.  An entry
+ * outside [0, Lv) copies row p instead and is reported as SVG_ERR_INVALID_ARG
+ * by svg_sync_status. */
 svg_status svg2_permute(const svg_shape* shape, const int32_t* perm_q, const int32_t* perm_k, const uint16_t* q,
                         const uint16_t* k, const uint16_t* v, uint16_t* q_out, uint16_t* k_out, uint16_t* v_out,
                         void* stream);
@@ -306,7 +309,9 @@ svg_status svg2_build_block_index(const svg_shape* shape, const svg_params* para
 
 /* Block-sparse attention in cluster order (q, k, v from svg2_permute) with the
  * cluster mask, written back in model order: video position p goes to row
- * perm_q[p] of out (and of lse_out, if given).  Requires block_q = 128. */
+ * perm_q[p] of out (and of lse_out, if given).  Requires block_q = 128.  A
+ * perm_q entry outside [0, Lv) leaves its row unwritten and is reported as
+ * SVG_ERR_INVALID_ARG by svg_sync_status. */
 svg_status svg2_attention(const svg_shape* shape, const svg_params* params, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, int Cq, int Ck, const int32_t* qoff, const int32_t* koff,
                           const uint64_t* sel, const int32_t* perm_q, const int32_t* row_ptr, const int32_t* col,

@@ -85,7 +85,15 @@ template <bool CLUSTER>
 __device__ __forceinline__ int out_row(const AttnArgs& a, int kind, int bh, int row) {
   const Geometry& g = a.g;
   if (row >= g.Lv) return row;
-  if constexpr (CLUSTER) return a.out_perm[static_cast<int64_t>(bh) * g.Lv + row];
+  if constexpr (CLUSTER) {
+    // a caller's permutation: an entry outside [0, Lv) is reported and its row not written
+    const int p = __ldg(a.out_perm + static_cast<int64_t>(bh) * g.Lv + row);
+    if (static_cast<unsigned>(p) >= static_cast<unsigned>(g.Lv)) {
+      atomicOr(&g_error_word, kErrBadIndex);
+      return -1;
+    }
+    return p;
+  }
   if (!a.model_order || kind != SVG_HEAD_TEMPORAL) return row;
   const int s = row / g.F, f = row - s * g.F;
   return f * g.S + s;

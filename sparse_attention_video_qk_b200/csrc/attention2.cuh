@@ -338,8 +338,8 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
             const int vend = min(k0 + 32, g.Lv);
             if (k0 < vend) {
               int jc = cluster_of(ko, a.Ck, k0);          // ko[jc] <= s0 < ko[Ck] = Lv
-              for (int s0 = k0; s0 < vend; jc++) {
-                const int e = min(__ldg(ko + jc + 1), vend);
+              for (int s0 = k0; s0 < vend && jc < a.Ck; jc++) {
+                const int e = max(s0, min(__ldg(ko + jc + 1), vend));   // max: a malformed table cannot move back
                 if ((rmask >> jc) & 1ull) keep |= span_bits(s0 - k0, e - k0);
                 s0 = e;
               }
@@ -474,14 +474,16 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
     if (ok && nT > 0 && __all_sync(0xffffffffu, mbar_wait(b_o(w), (nT - 1) & 1, abort_flag))) {
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row<CLUSTER>(a, kind, bh, row);
+      const int orow_t = row_ok ? out_row<CLUSTER>(a, kind, bh, row) : 0;
+      const bool write = row_ok && orow_t >= 0;
+      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + orow_t;
       uint16_t* orow = a.out + orow_i * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; c++) {
         uint32_t o[32];
         tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();
-        if (row_ok) {
+        if (write) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int v = 0; v < 4; v++) {
@@ -494,12 +496,15 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
           }
         }
       }
-      if (row_ok && a.lse) a.lse[orow_i] = (l > 0.f) ? (m_use * 0.69314718055994531f + logf(l)) : -INFINITY;
+      if (write && a.lse) a.lse[orow_i] = (l > 0.f) ? (m_use * 0.69314718055994531f + logf(l)) : -INFINITY;
     } else if (ok && nT == 0 && row_ok) {
-      const int64_t orow_i = static_cast<int64_t>(bh) * g.L + out_row<CLUSTER>(a, kind, bh, row);
-      uint4* dst = reinterpret_cast<uint4*>(a.out + orow_i * D);
-      for (int v = 0; v < D / 8; v++) dst[v] = make_uint4(0, 0, 0, 0);
-      if (a.lse) a.lse[orow_i] = -INFINITY;
+      const int orow_t = out_row<CLUSTER>(a, kind, bh, row);
+      if (orow_t >= 0) {
+        const int64_t orow_i = static_cast<int64_t>(bh) * g.L + orow_t;
+        uint4* dst = reinterpret_cast<uint4*>(a.out + orow_i * D);
+        for (int v = 0; v < D / 8; v++) dst[v] = make_uint4(0, 0, 0, 0);
+        if (a.lse) a.lse[orow_i] = -INFINITY;
+      }
     }
   }
   tc_fence_before();

@@ -293,7 +293,12 @@ __global__ void __launch_bounds__(1024) km_perm_kernel(const uint8_t* __restrict
   // cluster sizes -> first positions
   if (tid <= kMaxClusters) base[tid] = 0;
   __syncthreads();
-  for (int r = tid; r < Lv; r += 1024) atomicAdd(&base[as[r] + 1], 1);
+  // a cluster id outside [0, C) (a caller's assignment) is reported and its row left out
+  for (int r = tid; r < Lv; r += 1024) {
+    const int c = as[r];
+    if (c < C) atomicAdd(&base[c + 1], 1);
+    else atomicOr(&g_error_word, kErrBadIndex);
+  }
   __syncthreads();
   if (tid == 0) {
     for (int c = 0; c < C; c++) base[c + 1] += base[c];
@@ -302,7 +307,7 @@ __global__ void __launch_bounds__(1024) km_perm_kernel(const uint8_t* __restrict
   __syncthreads();
   for (int r0 = 0; r0 < Lv; r0 += 1024) {
     const int r = r0 + tid;
-    const int c = (r < Lv) ? as[r] : -1;
+    const int c = (r < Lv && as[r] < C) ? as[r] : -1;
     const unsigned same = __match_any_sync(0xffffffffu, c);
     const int rank = __popc(same & ((1u << lane) - 1u));
     for (int i = tid; i < 32 * kMaxClusters; i += 1024) (&wcount[0][0])[i] = 0;
@@ -415,7 +420,11 @@ __global__ void __launch_bounds__(256) km_gather_kernel(const KmGatherArgs a) {
       if (i < n) {
         const int row = static_cast<int>(i >> SH), c = static_cast<int>(i & (CH - 1));
         const int bh = fdiv(row, a.divL), p = row - bh * a.L;
-        const int sp = (p < a.Lv) ? __ldg(perm + static_cast<int64_t>(bh) * a.Lv + p) : p;
+        int sp = (p < a.Lv) ? __ldg(perm + static_cast<int64_t>(bh) * a.Lv + p) : p;
+        if (p < a.Lv && static_cast<unsigned>(sp) >= static_cast<unsigned>(a.Lv)) {   // a caller's entry out of range
+          atomicOr(&g_error_word, kErrBadIndex);
+          sp = p;
+        }
         x[u] = __ldg(src + (static_cast<int64_t>(bh) * a.L + sp) * CH + c);
       }
     }

@@ -376,3 +376,32 @@ def test_layer_at_the_hunyuanvideo_shape_on_two_heads():
     want = oracle.attention2_rows(q2, k2, v2, wl.Lv, aq, ak, sel, rows)
     got = host_bits(out).reshape(wl.H, wl.L, wl.d)[heads].reshape(-1, wl.d)[rows]
     assert_attention_close(got, want, what="hunyuan")
+
+
+def test_bad_cluster_ids_and_permutation_entries_are_reported():
+    """Caller-supplied assignments and permutations out of range are reported
+    (SVG_ERR_INVALID_ARG through svg_sync_status), and nothing outside the
+    buffers is touched."""
+    wl, inp, qn, kn, ref = case("d128")
+    pb = pb_of(wl)
+    a = ref["aq"].copy()
+    a[0, 5] = 200                                         # cluster id >= C
+    svg.svg2_permutation(pb, dev(a), 8)
+    with pytest.raises(svg.SVGError) as e:
+        svg.sync_status()
+    assert e.value.status == 1
+    pq = ref["pq"].copy()
+    pq[1, 3] = wl.Lv + 1000                               # position outside the video rows
+    svg.svg2_permute(pb, dev(pq), dev(ref["pk"]), dev(qn), dev(kn), dev(inp["v"]))
+    with pytest.raises(svg.SVGError) as e:
+        svg.sync_status()
+    assert e.value.status == 1
+    qp, kp, vp = (dev(oracle.permute_rows(x, wl.Lv, ref[p])) for x, p in ((qn, "pq"), (kn, "pk"), (inp["v"], "pk")))
+    qoff, koff, sel = dev(ref["qoff"]), dev(ref["koff"]), dev(ref["sel"].view(np.int64))
+    rp, col, full = svg.svg2_block_index(pb, qoff, koff, sel)
+    out = torch.zeros_like(qp)
+    svg.svg2_attention(pb, qp, kp, vp, qoff, koff, sel, dev(pq), rp, col, full, out=out)
+    with pytest.raises(svg.SVGError) as e:
+        svg.sync_status()
+    assert e.value.status == 1
+    svg.sync_status()
