@@ -175,3 +175,21 @@ def test_block_list2_covers_exactly_the_kept_pairs():
                 assert (kb in listed) == bool(t.any())
                 if kb in listed:
                     assert listed[kb] == int(t.all())
+
+
+def test_permute_rows_is_a_row_permutation_and_its_inverse_restores():
+    """oracle.permute_rows: the identity changes nothing, text rows stay, every
+    video row appears once, and the inverse permutation (argsort) restores
+    the input bit for bit."""
+    q, k, v, Lv, L, d = _small(seed=12, S=10, F=3, T=4)
+    ident = np.tile(np.arange(Lv, dtype=np.int32), (2, 1))
+    assert np.array_equal(oracle.permute_rows(q, Lv, ident), q)
+    rng = np.random.Generator(np.random.PCG64(4))
+    perm = np.stack([rng.permutation(Lv) for _ in range(2)]).astype(np.int32)
+    p = oracle.permute_rows(q, Lv, perm)
+    assert np.array_equal(p[0, :, Lv:], q[0, :, Lv:])
+    for h in range(2):
+        assert np.array_equal(p[0, h, :Lv], q[0, h, perm[h]])
+        assert sorted(map(bytes, p[0, h, :Lv])) == sorted(map(bytes, q[0, h, :Lv]))
+    inv = np.argsort(perm, axis=1).astype(np.int32)
+    assert np.array_equal(oracle.permute_rows(p, Lv, inv), q)
