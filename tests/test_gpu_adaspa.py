@@ -33,6 +33,8 @@ CASES = {
     "batch2": (W.small_workload(B=2, d=128, H=2, F=3, Hs=8, Ws=8, T=5, seed=34), 0.7),
     # Wan 2.1 1.3B shape (sampled query tiles)
     "wan": (W.WAN, 0.9),
+    # d = 64 at the CogVideoX shape (sampled query tiles)
+    "cogvideox": (W.COGVIDEOX, 0.8),
 }
 SMALL = ("d128", "d64", "notext", "batch2")
 

@@ -39,6 +39,8 @@ CASES = {
     "onecluster": (W.small_workload(d=64, H=2, F=2, Hs=6, Ws=8, T=3, seed=25), 1, 1, 1, 0.5),
     # 64 clusters (a full 64-bit key set) at the Wan 2.1 1.3B shape
     "wan": (W.WAN, 64, 64, 2, 0.9),
+    # d = 64 at the CogVideoX shape: 48 heads, 226 text tokens, 32 + 48 clusters
+    "cogvideox": (W.COGVIDEOX, 32, 48, 2, 0.9),
 }
 FULL_ROWS = ("d128", "d64", "notext", "batch2", "onecluster")
 
