@@ -193,3 +193,43 @@ def test_permute_rows_is_a_row_permutation_and_its_inverse_restores():
         assert sorted(map(bytes, p[0, h, :Lv])) == sorted(map(bytes, q[0, h, :Lv]))
     inv = np.argsort(perm, axis=1).astype(np.int32)
     assert np.array_equal(oracle.permute_rows(p, Lv, inv), q)
+
+
+def test_block_list2_bounds_the_closed_form_kept_pair_count():
+    """Independent of the mask: the kept pairs, from the cluster sizes alone
+    (a video query of cluster i keeps the keys of its selected clusters and
+    the text keys; a text query keeps all L), lie between the area of the
+    tiles marked full and the area of the listed tiles.  One cluster with
+    its set selected lists every tile as full; empty sets without text list
+    nothing."""
+    q, k, v, Lv, L, d = _small(seed=14, S=30, F=4, T=7)
+    _, aq, nq = oracle.kmeans(q, Lv, 5, 2)
+    _, ak, nk = oracle.kmeans(k, Lv, 6, 2)
+    pq, _ = oracle.cluster_permutation(aq, 5)
+    pk, _ = oracle.cluster_permutation(ak, 6)
+    rng = np.random.Generator(np.random.PCG64(6))
+    sel = rng.integers(1, 1 << 6, size=(2, 5)).astype(np.uint64)
+    bq, bk = 32, 16
+    rp, col, full = oracle.block_list2(L, Lv, bq, bk, aq, ak, pq, pk, sel)
+    nqb = -(-L // bq)
+    for h in range(2):
+        kept = sum(int(nq[h, i]) * (sum(int(nk[h, j]) for j in range(6) if (int(sel[h, i]) >> j) & 1) + (L - Lv))
+                   for i in range(5)) + (L - Lv) * L
+        listed_area = full_area = 0
+        for qb in range(nqb):
+            rows = min(bq, L - qb * bq)
+            for e in range(rp[h * nqb + qb], rp[h * nqb + qb + 1]):
+                a = rows * min(bk, L - int(col[e]) * bk)
+                listed_area += a
+                full_area += a if full[e] else 0
+        assert full_area <= kept <= listed_area
+    one = np.zeros_like(aq)
+    ident = np.tile(np.arange(Lv, dtype=np.int32), (2, 1))
+    rp1, col1, full1 = oracle.block_list2(L, Lv, bq, bk, one, one, ident, ident, np.ones((2, 1), np.uint64))
+    nkb = -(-L // bk)
+    assert len(col1) == 2 * nqb * nkb and full1.all()
+    q0, k0, v0, Lv0, L0, _ = _small(seed=15, S=30, F=2, T=0)
+    _, a0, _ = oracle.kmeans(q0, Lv0, 3, 1)
+    p0, _ = oracle.cluster_permutation(a0, 3)
+    rp0, col0, _ = oracle.block_list2(L0, Lv0, bq, bk, a0, a0, p0, p0, np.zeros((2, 3), np.uint64))
+    assert len(col0) == 0 and (rp0 == 0).all()
