@@ -110,7 +110,7 @@ def lib():
             L.ora_block_list.argtypes = [sh, pr, vp, vp, vp, vp]
             ci = ctypes.c_int
             L.ora2_kmeans_init.argtypes = [vp, ci, i64, i64, ci, ci, vp]
-            L.ora2_assign.argtypes = [vp, ci, i64, i64, ci, ci, vp, vp]
+            L.ora2_assign.argtypes = [vp, ci, i64, i64, ci, ci, vp, vp, vp]
             L.ora2_update.argtypes = [vp, ci, i64, i64, ci, ci, vp, vp, vp]
             L.ora2_kmeans.argtypes = [vp, ci, i64, i64, ci, ci, ci, vp, vp, vp]
             L.ora2_permutation.argtypes = [vp, ci, i64, ci, vp, vp]
@@ -122,7 +122,7 @@ def lib():
             dbl = ctypes.c_double
             L.ora3_block_mass.argtypes = [ci, i64, ci, ci, ci, dbl, vp, vp, vp, i64, vp, vp]
             L.ora3_select.restype = i64
-            L.ora3_select.argtypes = [ci, i64, i64, ci, ci, vp, dbl, vp, vp, vp, i64]
+            L.ora3_select.argtypes = [ci, i64, i64, ci, ci, vp, dbl, vp, vp, vp, i64, vp]
             L.ora3_attention_rows.argtypes = [ci, i64, ci, ci, ci, dbl, vp, vp, vp, vp, vp, i64, vp, vp, vp]
             _lib = L
     return _lib
@@ -296,13 +296,17 @@ def kmeans_init(x, Lv: int, C: int) -> np.ndarray:
     return cent
 
 
-def kmeans_assign(x, Lv: int, cent) -> np.ndarray:
+def kmeans_assign(x, Lv: int, cent, want_margin=False):
+    """Nearest centroid (fp64 squared distance) of every video row: uint8 [BH, Lv].
+    With want_margin also the per-row relative gap to the second nearest
+    centroid, (D2 - D1) / (|x|^2 + |c1|^2 + |c2|^2), float64 [BH, Lv]."""
     x = _c(x, np.uint16)
     cent = _c(cent, np.float32)
     BH, L, d = x.shape[0] * x.shape[1], x.shape[2], x.shape[3]
     out = np.empty((BH, Lv), np.uint8)
-    lib().ora2_assign(_ptr(x), BH, L, Lv, d, cent.shape[1], _ptr(cent), _ptr(out))
-    return out
+    margin = np.empty((BH, Lv), np.float64) if want_margin else None
+    lib().ora2_assign(_ptr(x), BH, L, Lv, d, cent.shape[1], _ptr(cent), _ptr(out), _ptr(margin))
+    return (out, margin) if want_margin else out
 
 
 def kmeans_update(x, Lv: int, assign, cent):
@@ -419,16 +423,21 @@ def block_mass(q, k, lse, bq: int, bk: int, scale=None, tiles=None):
     return mass
 
 
-def adaspa_select(mass, L: int, Lv: int, bq: int, bk: int, p: float):
-    """Kept key tiles from float32 masses [BH, nqb, nkb]: (row_ptr, col, full)."""
+def adaspa_select(mass, L: int, Lv: int, bq: int, bk: int, p: float, want_margin=False):
+    """Kept key tiles from float32 masses [BH, nqb, nkb]: (row_ptr, col, full).
+    With want_margin also each query tile's distance of its running sums from
+    the goal at the cut, float64 [BH*nqb] (+inf where nothing is cut)."""
     mass = _c(mass, np.float32)
     BH, nqb, nkb = mass.shape
     cap = BH * nqb * nkb
     row_ptr = np.empty(BH * nqb + 1, np.int32)
     col = np.empty(cap, np.int32)
     full = np.empty(cap, np.uint8)
-    n = lib().ora3_select(BH, L, Lv, bq, bk, _ptr(mass), float(p), _ptr(row_ptr), _ptr(col), _ptr(full), cap)
-    return row_ptr, col[:n], full[:n]
+    margin = np.empty(BH * nqb, np.float64) if want_margin else None
+    n = lib().ora3_select(BH, L, Lv, bq, bk, _ptr(mass), float(p), _ptr(row_ptr), _ptr(col), _ptr(full), cap,
+                          _ptr(margin))
+    res = (row_ptr, col[:n], full[:n])
+    return res + (margin,) if want_margin else res
 
 
 def block_attention_rows(q, k, v, bq: int, bk: int, row_ptr, col, rows, scale=None, want_lse=False):

@@ -20,9 +20,9 @@
  *   - head-adaptive: every head, and every query tile in it, keeps the
  *     smallest set of video key tiles, heaviest first, whose mass reaches p
  *     times the mass of all its video key tiles, so the density follows the
- *     head.  At least the heaviest video key tile is kept.  Masses are summed
- *     in 32-bit fixed point (mass * 2^32, truncated) so the running sums are
- *     exact and do not depend on their order; ties go to the lower tile index;
+ *     head.  At least the heaviest video key tile is kept.  The running sum and
+ *     the total are plain double sums of the masses in the heaviest-first order;
+ *     ties in mass go to the lower tile index;
  *   - hierarchical between modalities: key tiles holding text keys are kept
  *     by every query tile, and query tiles holding text rows keep every key
  *     tile, as in the rest of this library;
@@ -40,8 +40,6 @@ static double bf16_to_f64_3(uint16_t h) {
   memcpy(&f, &u, sizeof f);
   return (double)f;
 }
-
-#define ORA3_FIX 4294967296.0 /* 2^32 */
 
 /* Block masses.  Q, K: bf16 [BH][L][d]; lse: float [BH][L] (natural log).
  * mass[bh][qb][kb] = sum over rows q < L of tile qb and keys k < L of tile kb
@@ -73,11 +71,13 @@ void ora3_block_mass(int BH, int64_t L, int d, int bq, int bk, double scale, con
 
 /* Kept key tiles of every (head, query tile), from float masses
  * mass: float [BH][nqb][nkb].  Returns the entry count; row_ptr [BH*nqb+1],
- * col (increasing within a tile) and full (all 1) written up to `capacity`. */
+ * col (increasing within a tile) and full (all 1) written up to `capacity`.
+ * margin (nullable): double [BH*nqb], how far the cut is from moving: the
+ * smaller of (goal - running sum before the last kept tile) and (running sum
+ * with it - goal); +inf where no cut is made (text rows, no video tiles). */
 int64_t ora3_select(int BH, int64_t L, int64_t Lv, int bq, int bk, const float* mass, double p,
-                    int32_t* row_ptr, int32_t* col, uint8_t* full, int64_t capacity) {
+                    int32_t* row_ptr, int32_t* col, uint8_t* full, int64_t capacity, double* margin) {
   int64_t nqb = (L + bq - 1) / bq, nkb = (L + bk - 1) / bk;
-  int64_t* fix = (int64_t*)malloc(sizeof(int64_t) * (size_t)nkb);
   int* order = (int*)malloc(sizeof(int) * (size_t)nkb);
   uint8_t* keep = (uint8_t*)malloc((size_t)nkb);
   int64_t e = 0;
@@ -88,17 +88,13 @@ int64_t ora3_select(int BH, int64_t L, int64_t Lv, int bq, int bk, const float* 
     int64_t q1 = (qb + 1) * bq < L ? (qb + 1) * bq : L;
     int text_q = q1 > Lv;                       /* the tile holds a text row */
     int nv = 0;                                 /* video key tiles: every key of the tile < Lv */
-    int64_t total = 0;
     for (int64_t kb = 0; kb < nkb; kb++) {
       int64_t k1 = (kb + 1) * bk < L ? (kb + 1) * bk : L;
       int text_k = k1 > Lv;                     /* the tile holds a text key */
       keep[kb] = (uint8_t)(text_q || text_k);
-      if (!text_k) {
-        fix[kb] = (int64_t)((double)m[kb] * ORA3_FIX);
-        total += fix[kb];
-        order[nv++] = (int)kb;
-      }
+      if (!text_k) order[nv++] = (int)kb;
     }
+    if (margin) margin[t] = INFINITY;
     if (!text_q && nv > 0) {
       /* insertion sort of the video tiles: mass descending, lower index first */
       for (int a = 1; a < nv; a++) {
@@ -109,14 +105,17 @@ int64_t ora3_select(int BH, int64_t L, int64_t Lv, int bq, int bk, const float* 
         }
         order[b + 1] = x;
       }
+      double total = 0.0;
+      for (int a = 0; a < nv; a++) total += (double)m[order[a]];
       /* the heaviest tile, then more until the running sum reaches the goal */
-      double goal = p * (double)total;
-      int64_t run = 0;
+      double goal = p * total, run = 0.0, before = 0.0;
       for (int a = 0; a < nv; a++) {
         keep[order[a]] = 1;
-        run += fix[order[a]];
-        if ((double)run >= goal) break;
+        before = run;
+        run += (double)m[order[a]];
+        if (run >= goal) break;
       }
+      if (margin) margin[t] = fmin(goal - before, run - goal);
     }
     for (int64_t kb = 0; kb < nkb; kb++)
       if (keep[kb]) {
@@ -128,7 +127,6 @@ int64_t ora3_select(int BH, int64_t L, int64_t Lv, int bq, int bk, const float* 
       }
     row_ptr[t + 1] = (int32_t)e;
   }
-  free(fix);
   free(order);
   free(keep);
   return e;

@@ -18,22 +18,20 @@
  *   4. attention of each query row to the keys of its selected clusters.
  * The page gives no numbers or precisions.  Readings (also in the design notes):
  *   - init: centroid c = row floor(c * Lv / C); text rows are not clustered;
- *   - the nearest centroid minimises |c|^2 - 2 x.c (the squared Euclidean
- *     distance without the |x|^2 term, which is the same for every centroid);
- *     |c|^2 and x.c are each accumulated in float in the order i = 0..d-1 with
- *     fused multiply-add, then |c|^2 - 2 (x.c) is rounded once; the lowest
- *     index wins a tie.  This decides an integer, so it is taken in the
- *     precision the kernel uses;
- *   - a centroid sum is kept in 64-bit fixed point (value * 2^40, truncated
- *     toward zero), so its value does not depend on the order of the rows; the
- *     mean is ((double)sum / 2^40) / count rounded to float; an empty cluster
- *     keeps its centroid;
+ *   - the nearest centroid minimises the squared Euclidean distance
+ *     sum_i (x_i - c_i)^2, evaluated in double; the lowest index wins a tie;
+ *   - a centroid is the mean of its rows: the sum in double over the rows in
+ *     their order, divided by the count, rounded once to float; an empty
+ *     cluster keeps its centroid;
  *   - the permutation is a stable counting sort by cluster;
  *   - score s_ij = scale * (c^q_i . c^k_j) in double; weight
  *     w_ij = n^k_j * exp(s_ij - max_j s_ij); key clusters sorted by weight
  *     (descending, lower index first on a tie); the selected set is the
  *     shortest prefix whose running sum reaches p * (sum of all weights);
  *   - text keys are kept for every query and text queries keep every key.
+ * A library that takes the nearest-centroid decision in float may disagree
+ * with this one where the two nearest centroids are almost equally far; the
+ * assignment can report, per row, how far the decision is from such a tie.
  */
 #include <math.h>
 #include <stdint.h>
@@ -54,8 +52,6 @@ static float bf16_to_f32(uint16_t h) {
   return f;
 }
 
-#define ORA2_FIX 1099511627776.0   /* 2^40 */
-
 /* Centroid c = row floor(c * Lv / C) of the head, as float.
  * x: bf16 [BH][L][d]; cent: float [BH][C][d]. */
 void ora2_kmeans_init(const uint16_t* x, int BH, int64_t L, int64_t Lv, int d, int C, float* cent) {
@@ -66,50 +62,68 @@ void ora2_kmeans_init(const uint16_t* x, int BH, int64_t L, int64_t Lv, int d, i
     }
 }
 
-/* Nearest centroid of every video row (step 1, assignment).  assign: uint8 [BH][Lv]. */
+/* Nearest centroid of every video row (step 1, assignment).  assign: uint8
+ * [BH][Lv].  margin (nullable): double [BH][Lv], the gap between the second
+ * nearest and the nearest squared distance over |x|^2 + |c1|^2 + |c2|^2 (the
+ * scale of the terms a distance is formed from); +inf with one centroid. */
 void ora2_assign(const uint16_t* x, int BH, int64_t L, int64_t Lv, int d, int C, const float* cent,
-                 uint8_t* assign) {
+                 uint8_t* assign, double* margin) {
 #pragma omp parallel for schedule(static)
   for (int64_t g = 0; g < (int64_t)BH * Lv; g++) {
     int64_t bh = g / Lv, r = g % Lv;
     const uint16_t* xr = x + (bh * L + r) * d;
-    int best = 0;
-    float bestd = INFINITY;
+    int best = 0, second = -1;
+    double bestd = INFINITY, secondd = INFINITY;
     for (int c = 0; c < C; c++) {
       const float* cc = cent + (bh * C + c) * d;
-      float cn = 0.0f, dot = 0.0f;
+      double dist = 0.0;
       for (int i = 0; i < d; i++) {
-        cn = fmaf(cc[i], cc[i], cn);
-        dot = fmaf(bf16_to_f32(xr[i]), cc[i], dot);
+        double diff = bf16_to_f64(xr[i]) - (double)cc[i];
+        dist += diff * diff;
       }
-      const float dist = fmaf(-2.0f, dot, cn);
       if (dist < bestd) {
+        second = best;
+        secondd = bestd;
         bestd = dist;
         best = c;
+      } else if (dist < secondd) {
+        secondd = dist;
+        second = c;
       }
     }
     assign[g] = (uint8_t)best;
+    if (margin) {
+      if (second < 0) {
+        margin[g] = INFINITY;
+      } else {
+        double n = 0.0;
+        for (int i = 0; i < d; i++) {
+          double xi = bf16_to_f64(xr[i]), a = cent[(bh * C + best) * d + i], b = cent[(bh * C + second) * d + i];
+          n += xi * xi + a * a + b * b;
+        }
+        margin[g] = (secondd - bestd) / n;
+      }
+    }
   }
 }
 
 /* Centroids as the means of their rows (step 1, update); counts: int32 [BH][C]. */
 void ora2_update(const uint16_t* x, int BH, int64_t L, int64_t Lv, int d, int C, const uint8_t* assign,
                  float* cent, int32_t* counts) {
-  int64_t* sum = (int64_t*)calloc((size_t)C * d, sizeof(int64_t));
+  double* sum = (double*)calloc((size_t)C * d, sizeof(double));
   for (int bh = 0; bh < BH; bh++) {
-    memset(sum, 0, sizeof(int64_t) * (size_t)C * d);
+    memset(sum, 0, sizeof(double) * (size_t)C * d);
     for (int c = 0; c < C; c++) counts[bh * C + c] = 0;
     for (int64_t r = 0; r < Lv; r++) {
       int c = assign[(int64_t)bh * Lv + r];
       counts[bh * C + c]++;
       const uint16_t* xr = x + ((int64_t)bh * L + r) * d;
-      for (int i = 0; i < d; i++) sum[(int64_t)c * d + i] += (int64_t)(bf16_to_f64(xr[i]) * ORA2_FIX);
+      for (int i = 0; i < d; i++) sum[(int64_t)c * d + i] += bf16_to_f64(xr[i]);
     }
     for (int c = 0; c < C; c++) {
       int n = counts[bh * C + c];
       if (n == 0) continue;
-      for (int i = 0; i < d; i++)
-        cent[((int64_t)bh * C + c) * d + i] = (float)(((double)sum[(int64_t)c * d + i] / ORA2_FIX) / (double)n);
+      for (int i = 0; i < d; i++) cent[((int64_t)bh * C + c) * d + i] = (float)(sum[(int64_t)c * d + i] / (double)n);
     }
   }
   free(sum);
@@ -119,10 +133,10 @@ void ora2_update(const uint16_t* x, int BH, int64_t L, int64_t Lv, int d, int C,
 void ora2_kmeans(const uint16_t* x, int BH, int64_t L, int64_t Lv, int d, int C, int iters, float* cent,
                  uint8_t* assign, int32_t* counts) {
   for (int t = 0; t < iters; t++) {
-    ora2_assign(x, BH, L, Lv, d, C, cent, assign);
+    ora2_assign(x, BH, L, Lv, d, C, cent, assign, NULL);
     ora2_update(x, BH, L, Lv, d, C, assign, cent, counts);
   }
-  ora2_assign(x, BH, L, Lv, d, C, cent, assign);
+  ora2_assign(x, BH, L, Lv, d, C, cent, assign, NULL);
   /* the counts of the final assignment */
   for (int bh = 0; bh < BH; bh++) {
     for (int c = 0; c < C; c++) counts[bh * C + c] = 0;

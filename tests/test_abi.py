@@ -1,6 +1,7 @@
 """The C-ABI library loads, exports every declared symbol, and its host-side
 logic (argument checks, helpers) works without a GPU."""
 import ctypes
+import json
 import os
 import re
 
@@ -47,6 +48,38 @@ def test_sample_queries_matches_generator(L):
     assert sorted(out.tolist()) == list(range(50))          # n = Lv: a permutation
     with pytest.raises(C.SVGError):
         api.sample_queries(1, 10, 11)
+
+
+def _published_splitmix64():
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "splitmix64.json")
+    with open(path) as f:
+        cases = json.load(f)["cases"]
+    out = []
+    for c in cases:
+        xs = c.get("outputs") or [int(h, 16) for h in c["outputs_hex"]]
+        out.append((c["seed"], xs))
+    return out
+
+
+def test_splitmix64_stream_equals_published_outputs():
+    """The generator module's SplitMix64 against published output sequences
+    (seed 0 of the reference implementation; seed 1234567 of the Rosetta Code
+    task): a change to any of its three constants or shifts fails here."""
+    for seed, xs in _published_splitmix64():
+        gen = W.splitmix64_stream(seed)
+        assert [next(gen) for _ in xs] == xs, seed
+
+
+def test_sample_queries_c_helper_follows_published_outputs(L):
+    """The C helper's draws against the published SplitMix64 outputs.  With
+    Lv = 2^31 - 1 and n = 5 no slot is touched twice, so slot i receives
+    i + (x_(i+1) mod (Lv - i)) from the partial Fisher-Yates shuffle."""
+    Lv = (1 << 31) - 1
+    for seed, xs in _published_splitmix64():
+        want = [i + x % (Lv - i) for i, x in enumerate(xs)]
+        assert len(set(want)) == len(want) and min(want) >= len(xs)
+        assert api.sample_queries(seed, Lv, len(xs)).tolist() == want, seed
+        assert W.sample_queries(seed, Lv, len(xs)).tolist() == want, seed
 
 
 def test_rope_table_values(L):

@@ -4,7 +4,10 @@ the oracle, through the C ABI.
 Bars:
   * block masses: |gpu - oracle| <= 2e-4 * oracle + 1e-6 * (rows of the tile)
     (fp32 scores on the tensor cores, the hardware 2^x, fp32 sums);
-  * selection on the same float masses: bit-exact CSR;
+  * selection on the same float masses: bit-exact per query tile, except on
+    tiles whose cut lies within the kernel's fixed-point rounding of the goal
+    (the kernel sums trunc(mass * 2^32); the oracle sums in double), counted
+    and reported;
   * attention over a block list: max-abs 2e-2, mean-abs 2e-3 against fp64;
   * the whole search on the GPU: its selection equals the oracle's on every
     query tile whose decision is clear of the mass tolerance.
@@ -110,18 +113,39 @@ def test_block_mass_against_fp64(key):
         assert np.allclose(got.reshape(-1, wl.nqb, wl.nkb).sum(-1), rows[None, :], rtol=1e-3)
 
 
+def assert_select_matches(rp, col, full, m32, wl, p, what):
+    """The GPU's CSR selection against the oracle's on the same float masses.
+    The kernel sums the masses as trunc(mass * 2^32), so its running sums and
+    its goal are each off by less than (tiles) * 2^-32: a query tile whose
+    oracle running sum lies closer than 2 * nkb * 2^-32 to the goal at the cut
+    may be cut one tile earlier or later.  Every other tile is bit-exact."""
+    rp = rp.cpu().numpy() if hasattr(rp, "cpu") else rp
+    n = int(rp[-1])
+    col = (col.cpu().numpy() if hasattr(col, "cpu") else col)[:n]
+    full = (full.cpu().numpy() if hasattr(full, "cpu") else full)[:n]
+    rp_r, col_r, full_r, margin = oracle.adaspa_select(m32, wl.L, wl.Lv, wl.bq, wl.bk, p, want_margin=True)
+    band = 2 * wl.nkb * 2.0 ** -32
+    tie = margin < band
+    differ = 0
+    for t in range(len(rp) - 1):
+        same = col[rp[t]:rp[t + 1]].tolist() == col_r[rp_r[t]:rp_r[t + 1]].tolist()
+        if not same:
+            assert tie[t], f"{what}: query tile {t} differs outside the band (margin {margin[t]:.3e})"
+            differ += 1
+    assert (full == 1).all() and (full_r == 1).all()
+    print(f"{what}: {int(tie.sum())} of {len(tie)} query tiles in the band, {differ} differ")
+    assert tie.sum() <= 1e-3 * len(tie) + 2, what
+    if differ == 0:
+        assert np.array_equal(rp, rp_r) and np.array_equal(col, col_r)
+
+
 @pytest.mark.parametrize("key", SMALL)
-def test_select_bit_exact_on_the_same_masses(key):
+def test_select_matches_the_oracle_on_the_same_masses(key):
     wl, p, inp, qn, kn, lse, tiles, mass = case(key)
     m32 = mass.astype(np.float32).reshape(wl.B * wl.H, wl.nqb, wl.nkb)
     rp, col, full = svg.adaspa_select(pb_of(wl), dev(m32), p)
     svg.sync_status()
-    rp = rp.cpu().numpy()
-    n = int(rp[-1])
-    rp_r, col_r, full_r = oracle.adaspa_select(m32, wl.L, wl.Lv, wl.bq, wl.bk, p)
-    assert np.array_equal(rp, rp_r)
-    assert np.array_equal(col.cpu().numpy()[:n], col_r)
-    assert np.array_equal(full.cpu().numpy()[:n], full_r)
+    assert_select_matches(rp, col, full, m32, wl, p, key)
 
 
 def test_select_with_a_tight_capacity_matches():
@@ -140,7 +164,10 @@ def test_select_with_a_tight_capacity_matches():
 
 @pytest.mark.parametrize("p", [0.3, 0.6, 0.99, 1.0])
 def test_select_bit_exact_random_masses_with_ties(p):
-    """Masses with exact ties and zeros, over several sort sizes."""
+    """Masses with exact ties and zeros, over several sort sizes.  Multiples
+    of 1/8 are exact in both the kernel's fixed point and the oracle's double
+    sums, so every tile is bit-exact, on the band too (a running sum that meets
+    the goal exactly is a decision both sides take the same way)."""
     wl = W.small_workload(d=64, H=3, F=6, Hs=10, Ws=13, T=40, seed=2)   # nkb = 13
     rng = np.random.Generator(np.random.PCG64(int(p * 100)))
     m = rng.integers(0, 6, (wl.B * wl.H, wl.nqb, wl.nkb)).astype(np.float32) / 8

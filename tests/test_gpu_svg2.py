@@ -2,8 +2,13 @@
 "A. 语义感知排列" and "B. 基于质心的 Top-p 选择") with the oracle, through the C ABI.
 
 Bars:
-  * k-means centroids (float bits), assignments, cluster sizes, the cluster
-    sort, the permuted tensors and the block index: bit-exact;
+  * k-means, stage by stage on the same inputs: the initial centroids are
+    bit-exact; every assignment equals the oracle's fp64 nearest centroid
+    except on rows whose two nearest centroids lie within the tie band
+    (relative gap below 1e-5; the kernel takes the decision in fp32), and
+    those rows are counted and reported; every update is within one float
+    ulp of the fp64 mean;
+  * the cluster sort, the permuted tensors and the block index: bit-exact;
   * top-p sets: bit-exact wherever the oracle's weights leave the decision
     clear of a rounding-level near tie (the kernel's exp and the C library's
     may differ in the last bit);
@@ -99,31 +104,106 @@ def host(t):
 
 # --------------------------------------------------------------- k-means
 
+# The kernel decides the nearest centroid by |c|^2 - 2 x.c in fp32 (d-term
+# fused multiply-add chains), whose rounding error stays below about
+# d * 2^-24 * (|x|^2 + |c|^2) ~ 8e-6 of the terms' scale at d = 128.  A row
+# whose two nearest fp64 distances differ by less than TIE_BAND of
+# |x|^2 + |c1|^2 + |c2|^2 may therefore go either way.
+TIE_BAND = 1e-5
+
+
+def ordered_f32(bits):
+    """Monotone integer image of float32 bit patterns (adjacent floats differ by 1)."""
+    b = bits.astype(np.int64)
+    return np.where(b & 0x80000000, -(b & 0x7FFFFFFF), b)
+
+
+def check_assignment(x, Lv, cent, assign, what):
+    """The GPU assignment against the oracle's fp64 argmin under the same
+    centroids.  Returns (rows in the tie band, rows that differ)."""
+    want, margin = oracle.kmeans_assign(x, Lv, cent, want_margin=True)
+    diff = assign != want
+    tie = margin < TIE_BAND
+    assert not (diff & ~tie).any(), f"{what}: {(diff & ~tie).sum()} rows differ outside the tie band"
+    return int(tie.sum()), int(diff.sum())
+
+
+def check_update(x, Lv, assign_prev, cent_prev, cent, what):
+    """The GPU centroids against the oracle's fp64 means of the same assignment."""
+    want, _ = oracle.kmeans_update(x, Lv, assign_prev, cent_prev)
+    ulps = np.abs(ordered_f32(f32_bits(cent)) - ordered_f32(f32_bits(want)))
+    assert ulps.max() <= 1, f"{what}: centroids {ulps.max()} ulps from the fp64 mean"
+
+
+def kmeans_checked(pb, x, Lv, C, iters, what, cent0=None):
+    """The GPU k-means checked stage by stage against the oracle: each round is
+    one call warm-started from the previous call's centroids, so every
+    assignment and update is compared on the same inputs.  The single call of
+    `iters` rounds must equal the chain bit for bit.  Returns that call's
+    (cent, assign, counts) as numpy and the tie-band statistics."""
+    xd = dev(x)
+    stats = {"rows": 0, "tie_band": 0, "differ": 0}
+
+    def tally(t, dif):
+        stats["rows"] += int(np.prod(x.shape[:2])) * Lv
+        stats["tie_band"] += t
+        stats["differ"] += dif
+
+    if cent0 is None:
+        c, a, n = svg.svg2_kmeans(pb, xd, C, 0)
+        c_prev = oracle.kmeans_init(x, Lv, C)
+        assert np.array_equal(f32_bits(host(c)), f32_bits(c_prev)), f"{what}: initial centroids"
+    else:
+        c_prev = np.array(cent0, np.float32)
+        c, a, n = svg.svg2_kmeans(pb, xd, C, 0, cent=dev(c_prev))
+    a_prev = host(a)
+    tally(*check_assignment(x, Lv, c_prev, a_prev, f"{what} round 0"))
+    for t in range(1, iters + 1):
+        c, a, n = svg.svg2_kmeans(pb, xd, C, 1, cent=dev(c_prev))
+        c_h, a_h = host(c), host(a)
+        check_update(x, Lv, a_prev, c_prev, c_h, f"{what} round {t}")
+        tally(*check_assignment(x, Lv, c_h, a_h, f"{what} round {t}"))
+        c_prev, a_prev = c_h, a_h
+    c1, a1, n1 = svg.svg2_kmeans(pb, xd, C, iters, cent=None if cent0 is None else dev(np.array(cent0, np.float32)))
+    svg.sync_status()
+    c1, a1, n1 = host(c1), host(a1), host(n1)
+    assert np.array_equal(f32_bits(c1), f32_bits(c_prev)) and np.array_equal(a1, a_prev), f"{what}: one call != chain"
+    assert np.array_equal(n1, np.stack([np.bincount(r, minlength=C) for r in a1])), f"{what}: sizes"
+    print(f"{what}: {stats['tie_band']} of {stats['rows']} row decisions in the tie band, {stats['differ']} differ")
+    assert stats["tie_band"] <= 1e-4 * stats["rows"] + 2, f"{what}: {stats}"
+    return (c1, a1, n1), stats
+
+
 @pytest.mark.parametrize("key", list(CASES))
-def test_kmeans_bit_exact(key):
+def test_kmeans_matches_the_oracle_outside_the_tie_band(key):
     wl, inp, qn, kn, ref = case(key)
     _, Cq, Ck, iters, _ = CASES[key]
     pb = pb_of(wl)
     for x, C, s in ((qn, Cq, "q"), (kn, Ck, "k")):
-        cent, assign, counts = svg.svg2_kmeans(pb, dev(x), C, iters)
-        svg.sync_status()
-        assert np.array_equal(f32_bits(host(cent)), f32_bits(ref["c" + s])), f"{key}/{s}: centroids"
-        assert np.array_equal(host(assign), ref["a" + s]), f"{key}/{s}: assignment"
-        assert np.array_equal(host(counts), ref["n" + s]), f"{key}/{s}: sizes"
+        (cent, assign, counts), st = kmeans_checked(pb, x, wl.Lv, C, iters, f"{key}/{s}")
+        if st["differ"] == 0:
+            # no decision went the other way: the whole run equals the oracle's
+            ulps = np.abs(ordered_f32(f32_bits(cent)) - ordered_f32(f32_bits(ref["c" + s])))
+            assert ulps.max() <= 1 and np.array_equal(assign, ref["a" + s]), f"{key}/{s}"
+            assert np.array_equal(counts, ref["n" + s]), f"{key}/{s}: sizes"
 
 
 def test_kmeans_warm_start_continues_the_iteration():
     """Two calls of one round each from the previous centroids (the cached
-    centroids of the pages) equal one call of two rounds."""
+    centroids of the pages) equal one call of two rounds; the rounds are
+    checked against the oracle from the given centroids."""
     wl, inp, qn, kn, ref = case("d128")
     pb = pb_of(wl)
     x = dev(kn)
     cent, _, _ = svg.svg2_kmeans(pb, x, 11, 1)
     cent, assign, counts = svg.svg2_kmeans(pb, x, 11, 1, cent=cent)
+    c2, a2, n2 = svg.svg2_kmeans(pb, x, 11, 2)
     svg.sync_status()
-    assert np.array_equal(f32_bits(host(cent)), f32_bits(ref["ck"]))
-    assert np.array_equal(host(assign), ref["ak"])
-    assert np.array_equal(host(counts), ref["nk"])
+    assert np.array_equal(f32_bits(host(cent)), f32_bits(host(c2)))
+    assert np.array_equal(host(assign), host(a2))
+    assert np.array_equal(host(counts), host(n2))
+    start = oracle.kmeans(kn, wl.Lv, 11, 1)[0]
+    kmeans_checked(pb, kn, wl.Lv, 11, 2, "warm start", cent0=start)
 
 
 def test_kmeans_zero_iterations_is_the_init_assignment():
@@ -133,7 +213,7 @@ def test_kmeans_zero_iterations_is_the_init_assignment():
     svg.sync_status()
     c_ref = oracle.kmeans_init(qn, wl.Lv, 7)
     assert np.array_equal(f32_bits(host(cent)), f32_bits(c_ref))
-    assert np.array_equal(host(assign), oracle.kmeans_assign(qn, wl.Lv, c_ref))
+    check_assignment(qn, wl.Lv, c_ref, host(assign), "init")
 
 
 # ------------------------------------------------------------ cluster sort
@@ -294,25 +374,39 @@ def test_attention_one_cluster_equals_dense_kernel():
 
 # ------------------------------------------------------------ whole step
 
+def oracle_downstream(wl, qn, kn, cq, ck, aq, ak, nk, top_p):
+    """The oracle's steps after k-means, on given clusters."""
+    pq, qoff = oracle.cluster_permutation(aq, cq.shape[1])
+    pk, koff = oracle.cluster_permutation(ak, ck.shape[1])
+    sel, weight = oracle.select_top_p(cq, ck, nk, 1.0 / np.sqrt(wl.d), top_p, want_weight=True)
+    return dict(pq=pq, qoff=qoff, pk=pk, koff=koff, sel=sel, clear=clear_decisions(weight, top_p))
+
+
 @pytest.mark.parametrize("key", ["d128", "batch2", "wan"])
 def test_layer_end_to_end(key):
     """SVG2Layer (k-means, sort, top-p, permute, block index, attention) on
-    the CUDA path alone, every intermediate against the oracle."""
+    the CUDA path alone.  Its k-means equals the stage-checked k-means call;
+    every later intermediate equals the oracle's on those clusters."""
     wl, inp, qn, kn, ref = case(key)
     _, Cq, Ck, iters, top_p = CASES[key]
-    assert ref["clear"].all(), "a near tie in this case: pick another seed"
-    layer = svg.SVG2Layer(pb_of(wl), Cq, Ck, iters, top_p)
+    pb = pb_of(wl)
+    (cq, aq, nq), _ = kmeans_checked(pb, qn, wl.Lv, Cq, iters, f"{key}/q")
+    (ck, ak, nk), _ = kmeans_checked(pb, kn, wl.Lv, Ck, iters, f"{key}/k")
+    down = oracle_downstream(wl, qn, kn, cq, ck, aq, ak, nk, top_p)
+    assert down["clear"].all(), "a near tie in this case: pick another seed"
+    layer = svg.SVG2Layer(pb, Cq, Ck, iters, top_p)
     out = layer(dev(qn), dev(kn), dev(inp["v"]))
     svg.sync_status()
     last = layer.last
-    assert np.array_equal(f32_bits(host(layer.cq)), f32_bits(ref["cq"]))
-    assert np.array_equal(f32_bits(host(layer.ck)), f32_bits(ref["ck"]))
+    assert np.array_equal(f32_bits(host(layer.cq)), f32_bits(cq))
+    assert np.array_equal(f32_bits(host(layer.ck)), f32_bits(ck))
+    assert np.array_equal(host(last["assign_q"]), aq) and np.array_equal(host(last["assign_k"]), ak)
     for name in ("pq", "pk", "qoff", "koff"):
         gname = {"pq": "perm_q", "pk": "perm_k"}.get(name, name)
-        assert np.array_equal(host(last[gname]), ref[name]), name
-    assert np.array_equal(host(last["sel"]).view(np.uint64), ref["sel"])
+        assert np.array_equal(host(last[gname]), down[name]), name
+    assert np.array_equal(host(last["sel"]).view(np.uint64), down["sel"])
     rows = rows_of(key, wl)
-    want = oracle.attention2_rows(qn, kn, inp["v"], wl.Lv, ref["aq"], ref["ak"], ref["sel"], rows)
+    want = oracle.attention2_rows(qn, kn, inp["v"], wl.Lv, aq, ak, down["sel"], rows)
     assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], want, what=key)
 
 
@@ -349,9 +443,10 @@ def test_block_index_capacity_overflow_is_reported():
 def test_layer_at_the_hunyuanvideo_shape_on_two_heads():
     """The whole layer at the HunyuanVideo 720p shape (24 heads, 119,056
     tokens, 64 + 64 clusters), checked on one planted-spatial and one
-    planted-temporal head: centroids, sort and top-p bit-exact, attention on
-    sampled rows (every step is per head, so two heads of the oracle stand
-    for the launch)."""
+    planted-temporal head: k-means stage by stage against the oracle (tie band
+    as above), sort and top-p bit-exact on the layer's clusters, attention on
+    sampled rows (every step is per head, so two heads of the oracle stand for
+    the launch)."""
     wl = W.HUNYUAN
     inp = W.make_inputs(wl)
     sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
@@ -362,20 +457,22 @@ def test_layer_at_the_hunyuanvideo_shape_on_two_heads():
     svg.sync_status()
     heads = [0, 1]
     q2, k2, v2 = (np.ascontiguousarray(x[:, heads]) for x in (qn, kn, inp["v"]))
-    cq, aq, nq = oracle.kmeans(q2, wl.Lv, 64, 2)
-    ck, ak, nk = oracle.kmeans(k2, wl.Lv, 64, 2)
-    pq, qoff = oracle.cluster_permutation(aq, 64)
-    sel, weight = oracle.select_top_p(cq, ck, nk, 1.0 / np.sqrt(wl.d), 0.9, want_weight=True)
-    assert clear_decisions(weight, 0.9).all()
+    pb2 = svg.Problem.from_workload(wl, H=2)
+    (cq, aq, nq), _ = kmeans_checked(pb2, q2, wl.Lv, 64, 2, "hunyuan/q")
+    (ck, ak, nk), _ = kmeans_checked(pb2, k2, wl.Lv, 64, 2, "hunyuan/k")
+    # the layer's k-means over 24 heads equals the per-head calls
     assert np.array_equal(f32_bits(host(layer.cq)[heads]), f32_bits(cq))
     assert np.array_equal(f32_bits(host(layer.ck)[heads]), f32_bits(ck))
-    assert np.array_equal(host(layer.last["perm_q"])[heads], pq)
-    assert np.array_equal(host(layer.last["qoff"])[heads], qoff)
-    assert np.array_equal(host(layer.last["sel"]).view(np.uint64)[heads], sel)
+    assert np.array_equal(host(layer.last["assign_q"])[heads], aq)
+    down = oracle_downstream(wl, q2, k2, cq, ck, aq, ak, nk, 0.9)
+    assert down["clear"].all()
+    assert np.array_equal(host(layer.last["perm_q"])[heads], down["pq"])
+    assert np.array_equal(host(layer.last["qoff"])[heads], down["qoff"])
+    assert np.array_equal(host(layer.last["sel"]).view(np.uint64)[heads], down["sel"])
     rng = np.random.Generator(np.random.PCG64(3))
     toks = np.unique(np.concatenate([rng.choice(wl.L, 40, replace=False), np.arange(wl.L - 8, wl.L)]))
     rows = np.concatenate([h * wl.L + toks for h in range(2)]).astype(np.int64)
-    want = oracle.attention2_rows(q2, k2, v2, wl.Lv, aq, ak, sel, rows)
+    want = oracle.attention2_rows(q2, k2, v2, wl.Lv, aq, ak, down["sel"], rows)
     got = host_bits(out).reshape(wl.H, wl.L, wl.d)[heads].reshape(-1, wl.d)[rows]
     assert_attention_close(got, want, what="hunyuan")
 

@@ -79,13 +79,27 @@ def _kept(rp, col, t):
 
 
 def test_select_on_exact_binary_fractions():
-    # video tiles 0..3 with masses 1/8, 1/2, 1/4, 1/8 (fixed-point sums exact); no text
+    # video tiles 0..3 with masses 1/8, 1/2, 1/4, 1/8 (every running sum exact in double); no text
     m, L, Lv, bq, bk = _one_tile([0.125, 0.5, 0.25, 0.125], bq=16)
     for p, want in ((0.25, [1]), (0.5, [1]), (0.5001, [1, 2]), (0.75, [1, 2]), (0.76, [0, 1, 2]),
                     (0.875, [0, 1, 2]), (0.9, [0, 1, 2, 3]), (1.0, [0, 1, 2, 3])):
         rp, col, full = oracle.adaspa_select(m, L, Lv, bq, bk, p)
         assert _kept(rp, col, 0) == want, p
         assert (full == 1).all()
+
+
+def test_select_margin_is_the_distance_of_the_cut_from_the_goal():
+    """Sorted masses 1/2, 1/4, 1/8, 1/8 (total 1): at p = 0.7 the cut falls
+    after 1/2 + 1/4 = 0.75, so the margin is min(0.7 - 0.5, 0.75 - 0.7); at
+    p = 0.75 the running sum meets the goal exactly (margin 0); text query
+    tiles make no cut (+inf)."""
+    m, L, Lv, bq, bk = _one_tile([0.125, 0.5, 0.25, 0.125], text_cols=3, bq=16)
+    rp, col, full, margin = oracle.adaspa_select(m, L, Lv, bq, bk, 0.7, want_margin=True)
+    assert _kept(rp, col, 0)[:2] == [1, 2]
+    assert abs(margin[0] - 0.05) < 1e-15
+    assert np.isinf(margin[-1])                          # the last query tile holds the text rows
+    _, _, _, m2 = oracle.adaspa_select(m, L, Lv, bq, bk, 0.75, want_margin=True)
+    assert m2[0] == 0.0
 
 
 def test_select_keeps_text_keys_and_text_query_tiles_keep_all():

@@ -33,41 +33,49 @@ def test_kmeans_recovers_planted_clusters():
             assert np.allclose(cent[h, c], mean, rtol=0, atol=1e-6)
 
 
-def test_assignment_is_the_nearest_centroid_away_from_ties():
+def test_assignment_is_the_fp64_argmin_on_every_row():
+    """The assignment is numpy's brute-force argmin of the squared Euclidean
+    distance on every row (no tie band: both sides are fp64), and the margin is
+    the relative gap to the second nearest centroid."""
     rng = np.random.Generator(np.random.PCG64(5))
     x = W.to_bf16_bits(rng.standard_normal((1, 2, 200, 32)).astype(np.float32))
     cent = oracle.kmeans_init(x, 200, 7)
-    a = oracle.kmeans_assign(x, 200, cent)
+    a, margin = oracle.kmeans_assign(x, 200, cent, want_margin=True)
     xf = W.bf16_bits_to_f32(x[0]).astype(np.float64)
     for h in range(2):
-        dist = ((xf[h][:, None, :] - cent[h][None].astype(np.float64)) ** 2).sum(-1)
-        srt = np.sort(dist, 1)
-        clear = (srt[:, 1] - srt[:, 0]) > 1e-4 * srt[:, 1]
-        assert clear.mean() > 0.95
-        assert np.array_equal(a[h][clear], dist.argmin(1)[clear])
-    # the init rows are rows floor(c*Lv/C)
+        c64 = cent[h].astype(np.float64)
+        dist = ((xf[h][:, None, :] - c64[None]) ** 2).sum(-1)
+        assert np.array_equal(a[h], dist.argmin(1))
+        order = np.argsort(dist, 1, kind="stable")
+        c1, c2 = order[:, 0], order[:, 1]
+        scale = (xf[h] ** 2).sum(1) + (c64[c1] ** 2).sum(1) + (c64[c2] ** 2).sum(1)
+        gap = (dist[np.arange(200), c2] - dist[np.arange(200), c1]) / scale
+        assert np.allclose(margin[h], gap, rtol=1e-9, atol=1e-15)
+    # the init rows are rows floor(c*Lv/C); each init row is its own centroid (distance 0)
     for c in range(7):
         assert np.array_equal(cent[1, c], W.bf16_bits_to_f32(x[0, 1, c * 200 // 7]))
+        assert a[1, c * 200 // 7] == c
 
 
-def test_update_is_the_mean_and_lloyd_does_not_increase_the_error():
-    rng = np.random.Generator(np.random.PCG64(9))
-    x = W.to_bf16_bits(rng.standard_normal((1, 1, 300, 16)).astype(np.float32))
-    xf = W.bf16_bits_to_f32(x[0, 0]).astype(np.float64)
-    cent = oracle.kmeans_init(x, 300, 5)
-    prev = np.inf
-    for _ in range(4):
-        a = oracle.kmeans_assign(x, 300, cent)
-        sse = ((xf - cent[0][a[0]].astype(np.float64)) ** 2).sum()
-        assert sse <= prev * (1 + 1e-6)
-        prev = sse
-        new, counts = oracle.kmeans_update(x, 300, a, cent)
-        for c in range(5):
-            if counts[0, c]:
-                assert np.allclose(new[0, c], xf[a[0] == c].mean(0), rtol=0, atol=2e-7)
-            else:
-                assert np.array_equal(new[0, c], cent[0, c])     # an empty cluster keeps its centroid
-        cent = new
+def test_assignment_tie_goes_to_the_lower_index_with_zero_margin():
+    """A row exactly halfway between two centroids: distance 1 to each of
+    +-e_0; the lower index wins and the margin is 0.  A third, farther
+    centroid does not change either."""
+    d = 8
+    x = np.zeros((1, 1, 3, d), np.float32)
+    x[0, 0, 1, 0] = 0.5                                  # nearer to +e_0
+    x[0, 0, 2, 1] = 4.0                                  # nearest to the third centroid
+    cent = np.zeros((1, 3, d), np.float32)
+    cent[0, 0, 0], cent[0, 1, 0], cent[0, 2, 1] = -1.0, 1.0, 3.0
+    a, margin = oracle.kmeans_assign(W.to_bf16_bits(x), 3, cent, want_margin=True)
+    assert a.tolist() == [[0, 1, 2]]
+    assert margin[0, 0] == 0.0
+    # row 1: distances 2.25 and 0.25 -> gap 2 over 0.25 + 1 + 1
+    assert margin[0, 1] == 2.0 / 2.25
+    # row 2: distances 1 (c2) and 17 (c0, c1) -> gap 16 over 16 + 9 + 1
+    assert margin[0, 2] == 16.0 / 26.0
+    one, m1 = oracle.kmeans_assign(W.to_bf16_bits(x), 3, cent[:, :1], want_margin=True)
+    assert one.tolist() == [[0, 0, 0]] and np.isinf(m1).all()
 
 
 def test_permutation_is_a_stable_cluster_sort():
