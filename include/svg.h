@@ -143,18 +143,25 @@ svg_status svg_profile_heads_raw_q(const svg_shape* shape, const svg_params* par
  * example a plugin running inside a host runtime that owns all device memory
  * and exposes no allocator, or a serving process that reserved its whole
  * memory pool at start-up and must not call cudaMalloc while serving.
- * It computes exactly what svg_profile_heads computes (same arguments minus
- * the workspace) and allocates nothing: its scratch is a fixed 16 MiB device
- * array inside the library, which every GPU that loads the library holds until
- * the process exits.
+ * It takes the same arguments as svg_profile_heads minus the workspace and
+ * allocates nothing: its scratch is a fixed 16 MiB device array inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  Its results are those of svg_profile_heads up to the order in which
+ * the key chunks are merged: when fewer chunks fit in the scratch than the
+ * workspace entry point uses, the MSEs may differ in their last bits (and a
+ * head whose two MSEs are that close may be given the other kind); with the
+ * same chunk count the results are bit-identical.
  *   - Size limit: one key chunk of partial results takes B*H*128*(3+2d)*4 bytes
  *     and the per-row error sums B*H*64*2*8 bytes; if together they exceed
  *     16 MiB (B*H > 125 at d=128, > 246 at d=64) the call returns
  *     SVG_ERR_CAPACITY and launches nothing.  Otherwise it splits the
  *     keys into as many chunks as fit (at most as many as svg_profile_heads).
  *   - Set-up: the first call on each device looks up the scratch's device
- *     address (cudaGetSymbolAddress, with that device current) and caches it;
- *     make that first call before any stream capture.
+ *     address (cudaGetSymbolAddress, with that device current) and caches it
+ *     for the life of the process; make that first call before any stream
+ *     capture.  The cache is never refreshed: after cudaDeviceReset on a
+ *     device the cached address is stale, so do not call this entry point on
+ *     that device again in the same process.
  *   - Sharing: every call uses the same scratch and leaves its contents behind.
  *     Each call writes every scratch entry it later reads, so nothing needs to
  *     start at zero; but two calls whose kernels overlap on the GPU (different
@@ -267,9 +274,13 @@ size_t svg2_kmeans_workspace_size(const svg_shape* shape, int C);
  * its centroid), then a final assignment.  The nearest centroid minimises
  * |c|^2 - 2 x.c (the squared distance less |x|^2): both sums in float with
  * fused multiply-add in the order i = 0..d-1, then |c|^2 - 2 (x.c) rounded
- * once; the lowest index wins a tie.  Sums in 64-bit fixed point (x * 2^40
- * truncated), exact while a cluster's sum of |x| stays below 2^23; mean
- * ((double)sum / 2^40) / count rounded to float.
+ * once; the lowest index wins a tie.  This equals the fp64 nearest centroid
+ * except where the two nearest squared distances differ by less than about
+ * 1e-5 of |x|^2 + |c1|^2 + |c2|^2.  Sums in 64-bit fixed point (x * 2^40
+ * truncated); mean ((double)sum / 2^40) / count rounded to float.  The sums
+ * are exact for |x| < min(2^23 / Lv, 2^12); a value outside that range (or
+ * inf / NaN) is left out of its sum and reported as SVG_ERR_INVALID_ARG by
+ * svg_sync_status.
  * cent: device float [B*H][C][d] (in/out); assign: device uint8 [B*H][Lv];
  * counts: device int32 [B*H][C], the sizes of the final assignment. */
 svg_status svg2_kmeans(const svg_shape* shape, const uint16_t* x, int C, int iters, int init, float* cent,
@@ -309,9 +320,10 @@ svg_status svg2_build_block_index(const svg_shape* shape, const svg_params* para
 
 /* Block-sparse attention in cluster order (q, k, v from svg2_permute) with the
  * cluster mask, written back in model order: video position p goes to row
- * perm_q[p] of out (and of lse_out, if given).  Requires block_q = 128.  A
- * perm_q entry outside [0, Lv) leaves its row unwritten and is reported as
- * SVG_ERR_INVALID_ARG by svg_sync_status. */
+ * perm_q[p] of out (and of lse_out, if given).  Requires block_q = 128.
+ * perm_q, qoff, koff and sel must not be NULL (SVG_ERR_INVALID_ARG before any
+ * launch).  A perm_q entry outside [0, Lv) leaves its row unwritten and is
+ * reported as SVG_ERR_INVALID_ARG by svg_sync_status. */
 svg_status svg2_attention(const svg_shape* shape, const svg_params* params, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, int Cq, int Ck, const int32_t* qoff, const int32_t* koff,
                           const uint64_t* sel, const int32_t* perm_q, const int32_t* row_ptr, const int32_t* col,

@@ -34,7 +34,16 @@ struct KmArgs {
   uint8_t* assign;         // [BH][Lv]
   int32_t* counts;         // [BH][C]
   unsigned long long* sum; // [BH][C][D] fixed-point sums
+  double xmax;             // values must satisfy |x| < xmax (km_value_bound)
 };
+
+// Largest |x| the fixed-point sums take exactly: a cluster of up to Lv rows
+// must keep its sum of |x| below 2^23 (x * 2^40 in a signed 64-bit word), and a
+// block's 2,048-row high-word sums must fit a signed 32-bit word (|x| < 2^12).
+__host__ __device__ inline double km_value_bound(int Lv) {
+  const double b = 8388608.0 / (Lv > 0 ? Lv : 1);
+  return b < 4096.0 ? b : 4096.0;
+}
 
 // Centroid c = video row floor(c * Lv / C) of the head.
 template <int D>
@@ -218,6 +227,7 @@ __global__ void __launch_bounds__(256) km_sum_kernel(const KmArgs a) {
 #pragma unroll
   for (int e = 0; e < E; e++) acc[e] = 0;
   int cur = -1;
+  bool out_of_range = false;
   auto flush = [&]() {
     if (cur < 0) return;
 #pragma unroll
@@ -250,11 +260,15 @@ __global__ void __launch_bounds__(256) km_sum_kernel(const KmArgs a) {
 #pragma unroll
       for (int e = 0; e < E; e++) {
         const double xd = static_cast<double>(__uint_as_float(static_cast<uint32_t>(xv[u][e]) << 16));
-        acc[e] += static_cast<long long>(xd * kFix);
+        // a value the sums cannot take exactly (or inf / NaN) is reported and left out
+        const bool ok = fabs(xd) < a.xmax;
+        out_of_range |= !ok;
+        acc[e] += ok ? static_cast<long long>(xd * kFix) : 0ll;
       }
     }
   }
   flush();
+  if (out_of_range) atomicOr(&g_error_word, kErrBadIndex);
   __syncthreads();
   unsigned long long* gs = a.sum + static_cast<int64_t>(bh) * n;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {

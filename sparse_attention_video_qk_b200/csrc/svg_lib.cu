@@ -630,6 +630,7 @@ svg_status svg2_kmeans(const svg_shape* s, const uint16_t* x, int C, int iters, 
   a.assign = assign;
   a.counts = counts;
   a.sum = static_cast<unsigned long long*>(workspace);
+  a.xmax = km_value_bound(Lv);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * a.BH * C, cs) != cudaSuccess) return SVG_ERR_CUDA;
   if (cudaMemsetAsync(workspace, 0, svg2_kmeans_workspace_size(s, C), cs) != cudaSuccess) return SVG_ERR_CUDA;
@@ -744,7 +745,7 @@ svg_status svg2_attention(const svg_shape* s, const svg_params* p, const uint16_
                           const uint16_t* v, int Cq, int Ck, const int32_t* qoff, const int32_t* koff,
                           const uint64_t* sel, const int32_t* perm_q, const int32_t* row_ptr, const int32_t* col,
                           const uint8_t* full, uint16_t* out, float* lse_out, void* stream) {
-  if (!qoff || !koff || !sel) return SVG_ERR_INVALID_ARG;
+  if (!qoff || !koff || !sel || !perm_q) return SVG_ERR_INVALID_ARG;
   if (Cq < 1 || Cq > kMaxClusters || Ck < 1 || Ck > kMaxClusters) return SVG_ERR_INVALID_ARG;
   AttnArgs c{};
   c.sel = sel;

@@ -145,6 +145,26 @@ def test_host_side_argument_errors(L):
                                None) == C.SVG_ERR_CAPACITY
 
 
+def test_svg2_attention_rejects_null_pointers(L):
+    """A NULL perm_q (or qoff, koff, sel) is an argument error returned before
+    any launch, not a device-side fault."""
+    pb = api.Problem.from_workload(W.small_workload(d=128, H=2, F=4, Hs=8, Ws=12, T=19))
+    sh, pr = pb.c_shape(), pb.c_params()
+    p = ctypes.c_void_p(16)
+    out = ctypes.c_void_p(16 + 4096)
+    for null in range(4):                       # qoff, koff, sel, perm_q
+        args = [p, p, p, p]
+        args[null] = None
+        qoff, koff, sel, perm_q = args
+        assert L.svg2_attention(ctypes.byref(sh), ctypes.byref(pr), p, p, p, 8, 11, qoff, koff, sel, perm_q, p, p, p,
+                                out, None, None) == C.SVG_ERR_INVALID_ARG, null
+    # through the binding too: None for perm_q raises before anything runs
+    with pytest.raises(C.SVGError) as e:
+        C.check(L.svg2_attention(ctypes.byref(sh), ctypes.byref(pr), p, p, p, 8, 11, p, p, p, None, p, p, p, out, None,
+                                 None), "svg2_attention")
+    assert e.value.status == C.SVG_ERR_INVALID_ARG
+
+
 def test_noalloc_capacity_limit(L):
     """The no-alloc profiling entry rejects shapes whose one key chunk of
     partials does not fit its 16 MiB scratch, before any CUDA call."""

@@ -302,6 +302,43 @@ def test_attention_hunyuan_sampled_rows():
     assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, "hunyuan")
 
 
+# ----------------------------------------------------------- sparsity sweep
+
+SWEEP = dict(W.sweep_points())
+
+
+@functools.lru_cache(maxsize=None)
+def sweep_case():
+    """Inputs of the sparsity sweep (the HunyuanVideo shape) and the oracle's
+    QK-Norm + RoPE of them; every sweep point shares them."""
+    wl = W.HUNYUAN_SWEEP
+    inp = W.make_inputs(wl)
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    return inp, oracle.qknorm_rope(sh, pr, inp["q"], inp["gamma_q"]), oracle.qknorm_rope(sh, pr, inp["k"],
+                                                                                            inp["gamma_k"])
+
+
+@pytest.mark.parametrize("point", list(SWEEP))
+def test_sparsity_sweep_point(point):
+    """Every point of the sparsity sweep at the HunyuanVideo 720p shape (all 24
+    heads forced to one kind; spatial windows 0-8 frames, temporal radii
+    32-1800): the block index bit-exact against the oracle's brute-force tile
+    list, and the attention launch bench.py times (layout, then attention with
+    the inverse layout in its epilogue) on sampled rows within 2e-2 / 2e-3."""
+    wl = SWEEP[point]
+    inp, qn, kn = sweep_case()
+    sh, pr = oracle.shape_of(wl), oracle.params_of(wl)
+    kinds = np.array(wl.forced_kinds, np.uint8)
+    rp, col, full = csr_host(*svg.build_block_index(pb_of(wl), dev(kinds)))
+    svg.sync_status()
+    rp_ref, col_ref, full_ref = oracle.block_list(sh, pr, kinds)
+    assert np.array_equal(rp, rp_ref) and np.array_equal(col, col_ref) and np.array_equal(full, full_ref), point
+    out, _ = run_sparse(wl, qn, kn, inp["v"], kinds, model_order=True)
+    rows = W.random_rows(wl, 32, seed=19, max_boundary_tiles=1)
+    ref = oracle.attention_rows(sh, pr, kinds, qn, kn, inp["v"], rows)
+    assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, point)
+
+
 # ---------------------------------------------------------------- full step
 
 @pytest.mark.parametrize("key,head_layout_out", [("tiny", False), ("smallS", False), ("batch2", False),

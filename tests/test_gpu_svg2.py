@@ -170,7 +170,10 @@ def kmeans_checked(pb, x, Lv, C, iters, what, cent0=None):
     assert np.array_equal(f32_bits(c1), f32_bits(c_prev)) and np.array_equal(a1, a_prev), f"{what}: one call != chain"
     assert np.array_equal(n1, np.stack([np.bincount(r, minlength=C) for r in a1])), f"{what}: sizes"
     print(f"{what}: {stats['tie_band']} of {stats['rows']} row decisions in the tie band, {stats['differ']} differ")
-    assert stats["tie_band"] <= 1e-4 * stats["rows"] + 2, f"{what}: {stats}"
+    # the band is a worst-case bound, so it holds a few rows per ten thousand; the
+    # decisions that actually went the other way must be rarer still
+    assert stats["tie_band"] <= 1e-3 * stats["rows"] + 2, f"{what}: {stats}"
+    assert stats["differ"] <= 1e-5 * stats["rows"] + 2, f"{what}: {stats}"
     return (c1, a1, n1), stats
 
 
@@ -422,6 +425,23 @@ def test_bad_arguments_are_reported():
     rp, col, full = svg.svg2_block_index(pb64, qoff, koff, sel)
     with pytest.raises(RuntimeError):
         svg.svg2_attention(pb64, dev(qn), dev(kn), dev(inp["v"]), qoff, koff, sel, dev(ref["pq"]), rp, col, full)
+    svg.sync_status()
+
+
+def test_kmeans_values_outside_the_exact_range_are_reported():
+    """A value the fixed-point centroid sums cannot hold exactly (here 1e30,
+    and a NaN) is left out and reported as SVG_ERR_INVALID_ARG; the next call
+    on clean inputs runs normally."""
+    wl, inp, qn, kn, ref = case("d128")
+    pb = pb_of(wl)
+    for bad in (0x7149, 0x7FC0):                      # bf16 bits of about 1e30, and a NaN
+        x = qn.copy()
+        x[0, 1, 7, 3] = bad
+        svg.svg2_kmeans(pb, dev(x), 8, 1)
+        with pytest.raises(svg.SVGError) as e:
+            svg.sync_status()
+        assert e.value.status == 1
+    cent, assign, counts = svg.svg2_kmeans(pb, dev(qn), 8, 0)
     svg.sync_status()
 
 
