@@ -51,6 +51,7 @@ struct Attn2Cfg {
   static __device__ __forceinline__ uint32_t tm_o(int w) { return 256u + static_cast<uint32_t>(D) * w; }
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(2 * NSLOT + 12 <= BAR_BYTES / 8, "barrier area");
+  static_assert(NSLOT >= 2, "a K and a V tile in flight");
 };
 
 // Walks the sorted union of two ascending CSR lists.  flags per list:
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
   }
   const int qb0 = 2 * pr, qb1 = 2 * pr + 1;          // qb1 may be past the last tile (empty list)
   const int ra0 = a.row_ptr[bh * g.nqb + qb0], ra1 = a.row_ptr[bh * g.nqb + qb0 + 1];
-  const int rb0 = (qb1 < g.nqb) ? ra1 : ra1, rb1 = (qb1 < g.nqb) ? a.row_ptr[bh * g.nqb + qb1 + 1] : ra1;
+  const int rb0 = ra1, rb1 = (qb1 < g.nqb) ? a.row_ptr[bh * g.nqb + qb1 + 1] : ra1;
 
   if (threadIdx.x == 0) {
     mbar_init(b_q, 1);
@@ -191,11 +192,19 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop (converged, so the descriptors stay in
+    // uniform registers); one elected lane issues each MMA and commit.
+    {
       constexpr uint32_t idS128 = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idS64 = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_base = smem_addr(sQ), kv_base = smem_addr(sKV);
+      // Descriptors of the operand bases.  An operand at byte offset o from a
+      // base has the base's descriptor plus o / 16: the start-address field holds
+      // address / 16 in 14 bits and every operand lies inside shared memory
+      // (< 256 KB), so the field never carries into the next one.
+      const uint64_t dq = sdesc_sw128(smem_addr(sQ), 16, 1024);
+      const uint64_t dk = sdesc_sw128(smem_addr(sKV), 16, 1024);
+      const uint64_t dv = sdesc_sw128(smem_addr(sKV), C::PANEL, 1024);
       UnionCursor cur{a.col, a.full, ra0, ra1, rb0, rb1};
       auto tile_blocks = [&]() {
         int kb, fa, fb, nb = 0;
@@ -203,68 +212,88 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
         if (nb == 1 && cur.next(kb, fa, fb)) nb = 2;
         return nb;
       };
-      auto issue_s = [&](int w, int j, int nb) {
-        const int st = (2 * j) % NSLOT;
+      // S_w = Q_w K^T: K = d in steps of 16 (32 bytes of a 128-byte swizzled row; 64 per panel)
+      auto issue_s = [&](int w, int st, int nb) {
+        const uint64_t a0 = dq + static_cast<uint32_t>((w * C::Q_BYTES) >> 4);
+        const uint64_t b0 = dk + static_cast<uint32_t>((st * C::SLOT_BYTES) >> 4);
+        const uint32_t id = nb == 2 ? idS128 : idS64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; kk++) {
-          const uint32_t off = (kk >> 2) * C::PANEL + (kk & 3) * 32;
-          umma_ss(tmem + C::tm_s(w), sdesc_sw128(q_base + w * C::Q_BYTES + off, 16, 1024),
-                  sdesc_sw128(kv_base + st * C::SLOT_BYTES + off, 16, 1024), nb == 2 ? idS128 : idS64, kk > 0);
+          const uint32_t o16 = static_cast<uint32_t>(((kk >> 2) * C::PANEL + (kk & 3) * 32) >> 4);
+          umma_ss_elect(tmem + C::tm_s(w), a0 + o16, b0 + o16, id, kk > 0);
         }
-        umma_commit(b_s(w));
+        umma_commit_elect(b_s(w));
       };
-      auto issue_pv = [&](int w, int j, int nb) {
-        const int st = (2 * j + 1) % NSLOT;
-        for (int kk = 0; kk < nb * 4; kk++) {
-          const uint64_t db = sdesc_sw128(kv_base + st * C::SLOT_BYTES + kk * 2048, C::PANEL, 1024);
-          umma_ts(tmem + C::tm_o(w), tmem + C::tm_s(w) + kk * 8, db, idO, (j > 0 || kk > 0) ? 1u : 0u);
+      // O_w += P_w V: K = keys in steps of 16 (2048 bytes of the MN-major V tile)
+      auto issue_pv = [&](int w, int st, int nb, bool first) {
+        const uint64_t b0 = dv + static_cast<uint32_t>((st * C::SLOT_BYTES) >> 4);
+        const uint32_t tp = tmem + C::tm_s(w), to = tmem + C::tm_o(w);
+        if (nb == 2) {
+#pragma unroll
+          for (int kk = 0; kk < 8; kk++) umma_ts_elect(to, tp + kk * 8, b0 + kk * (2048 >> 4), idO, (!first || kk > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; kk++) umma_ts_elect(to, tp + kk * 8, b0 + kk * (2048 >> 4), idO, (!first || kk > 0) ? 1u : 0u);
         }
-        umma_commit(b_o(w));
+        umma_commit_elect(b_o(w));
       };
+      // slot and phase of the ring entries: K of tile j is entry 2j, V entry 2j+1
+      int sk = 0, pk = 0;              // K of the current tile
+      auto advance = [&](int& st, int& ph) {
+        st += 2;
+        if (st >= NSLOT) {
+          st -= NSLOT;
+          ph ^= 1;
+        }
+      };
+      int sv = 1, pv = 0;              // V of the previous tile (entry 2j-1 at iteration j)
+      // every wait is made warp-uniform, so the warp stays converged for elect.sync
+      auto wait_all = [&](uint32_t bar, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(bar, par, abort_flag)); };
       bool issued_any = false;
-      bool ok = mbar_wait(b_q, 0, abort_flag);
+      bool ok = wait_all(b_q, 0);
       int nb_prev = 0;
       int nb = ok ? tile_blocks() : 0;
       if (ok && nb > 0) {
         // tile 0: S0, S1
-        if (!mbar_wait(b_full(0), 0, abort_flag)) ok = false;
+        if (!wait_all(b_full(sk), pk)) ok = false;
         if (ok) {
           tc_fence_after();
-          issue_s(0, 0, nb);
-          issue_s(1, 0, nb);
-          umma_commit(b_empty(0));
+          issue_s(0, sk, nb);
+          issue_s(1, sk, nb);
+          umma_commit_elect(b_empty(sk));
           issued_any = true;
         }
       }
       for (int j = 1; ok && nb > 0; j++) {
         nb_prev = nb;
         nb = tile_blocks();                       // blocks of tile j (0: no tile j)
-        const int iv = 2 * (j - 1) + 1;           // V of tile j-1
+        const int sv_prev = sv, pv_prev = pv;     // V of tile j-1
+        advance(sk, pk);                          // K of tile j
         // P.V0(j-1)
-        if (!mbar_wait(b_p(0), (j - 1) & 1, abort_flag)) break;
-        if (!mbar_wait(b_full(iv % NSLOT), (iv / NSLOT) & 1, abort_flag)) break;
+        if (!wait_all(b_p(0), (j - 1) & 1)) break;
+        if (!wait_all(b_full(sv_prev), pv_prev)) break;
         tc_fence_after();
-        issue_pv(0, j - 1, nb_prev);
+        issue_pv(0, sv_prev, nb_prev, j == 1);
         // S0(j)
-        const int ik = 2 * j;
         if (nb > 0) {
-          if (!mbar_wait(b_full(ik % NSLOT), (ik / NSLOT) & 1, abort_flag)) break;
+          if (!wait_all(b_full(sk), pk)) break;
           tc_fence_after();
-          issue_s(0, j, nb);
+          issue_s(0, sk, nb);
         }
         // P.V1(j-1)
-        if (!mbar_wait(b_p(1), (j - 1) & 1, abort_flag)) break;
+        if (!wait_all(b_p(1), (j - 1) & 1)) break;
         tc_fence_after();
-        issue_pv(1, j - 1, nb_prev);
-        umma_commit(b_empty(iv % NSLOT));
+        issue_pv(1, sv_prev, nb_prev, j == 1);
+        umma_commit_elect(b_empty(sv_prev));
         // S1(j)
         if (nb > 0) {
-          issue_s(1, j, nb);
-          umma_commit(b_empty(ik % NSLOT));
+          issue_s(1, sk, nb);
+          umma_commit_elect(b_empty(sk));
         }
+        advance(sv, pv);                          // V of tile j
       }
       if (*abort_flag && issued_any) {
-        umma_commit(b_drain);
+        umma_commit_elect(b_drain);
         mbar_wait_drain(b_drain, 0);
       }
     }
@@ -394,11 +423,8 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
       float m8[8];
 #pragma unroll
       for (int i = 0; i < 8; i++) m8[i] = -INFINITY;
-      if (j > 0) {
-        // one pass: exponentiate with the running maximum and track the tile's own maximum;
-        // the result stands unless the tile maximum outgrows the running one by 2^8
-        const float msub = (m_use == -INFINITY) ? 0.f : m_use;
-        const uint64_t nm2 = f32x2(-msub, -msub);
+      // A pass over the kept chunks of S; `body` sees each chunk with its mask applied.
+      auto pass = [&](auto&& body) {
 #pragma unroll
         for (int q = 0; q < 4; q++) {
           if (mode[q >> 1] == 2) {
@@ -408,22 +434,43 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
           }
           uint32_t v[32];
           load_chunk(q, v);
+          body(v, q);
+        }
+      };
+      bool rescale = (j == 0);
+      if (j > 0 && __all_sync(0xffffffffu, m_use != -INFINITY)) {
+        // Every row has a running maximum: exponentiate against it without tracking
+        // the tile's maximum.  The result stands while the tile's row sum of
+        // 2^(x - m) stays below 2^64: then no P exceeds 2^64, so P (bf16), l and O
+        // (fp32) stay far inside their range and keep their relative precision,
+        // however far m lags the true maximum.  Otherwise the tile's maximum is
+        // taken and the running one moves.
+        const uint64_t nm2 = f32x2(-m_use, -m_use);
+        pass([&](const uint32_t* v, int q) { chunk_exp(v, pk + 16 * q, acc, nm2); });
+        float s0, s1, s2, s3;
+        unpack2(acc[0], s0, s1);
+        unpack2(acc[1], s2, s3);
+        rescale = __any_sync(0xffffffffu, !(((s0 + s1) + (s2 + s3)) < 0x1p64f));
+        if (rescale) pass([&](const uint32_t* v, int q) { chunk_max(v, m8); });
+      } else if (j > 0) {
+        // some row has seen no kept key yet: exponentiate and track the maximum;
+        // the result stands unless it outgrows the running one by 2^8
+        const float msub = (m_use == -INFINITY) ? 0.f : m_use;
+        const uint64_t nm2 = f32x2(-msub, -msub);
+        pass([&](const uint32_t* v, int q) {
           chunk_max(v, m8);
           chunk_exp(v, pk + 16 * q, acc, nm2);
-        }
+        });
+        const float mxs = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
+        rescale = __any_sync(0xffffffffu, mxs > m_use + 8.0f);
       } else {
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-          if (mode[q >> 1] == 2) continue;
-          uint32_t v[32];
-          load_chunk(q, v);
-          chunk_max(v, m8);
-        }
+        // first tile: the running maximum starts at the tile's own
+        pass([&](const uint32_t* v, int q) { chunk_max(v, m8); });
       }
-      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-      const float mxs = mx * sl2;
-      const bool need_rescale = mxs > m_use + 8.0f;
-      if (j == 0 || __any_sync(0xffffffffu, need_rescale)) {
+      if (rescale) {
+        const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+        const float mxs = mx * sl2;
+        const bool need_rescale = mxs > m_use + 8.0f;
         const float m_new = need_rescale ? mxs : m_use;
         const float alpha = need_rescale ? ((m_use == -INFINITY) ? 0.f : fast_exp2(m_use - m_new)) : 1.f;
         l *= alpha;
@@ -446,17 +493,7 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
         const uint64_t nm2 = f32x2(-msub, -msub);
         acc[0] = 0ull;
         acc[1] = 0ull;
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-          if (mode[q >> 1] == 2) {
-#pragma unroll
-            for (int c = 0; c < 16; c++) pk[16 * q + c] = 0u;
-            continue;
-          }
-          uint32_t v[32];
-          load_chunk(q, v);
-          chunk_exp(v, pk + 16 * q, acc, nm2);
-        }
+        pass([&](const uint32_t* v, int q) { chunk_exp(v, pk + 16 * q, acc, nm2); });
       }
       // packed P over S columns [0, 64)
       tmem_st32(tS, pk);
