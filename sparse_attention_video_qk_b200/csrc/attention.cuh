@@ -125,29 +125,6 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-// 2^x of a packed pair on the FMA pipe (no exp unit), for x <= 126 (x may be
-// -inf).  x is clamped at -125 (2^-125 ~ 2.4e-38 stands for 0), split as
-// x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low bits) and
-// f in [-1/2, 1/2]; 2^f is a degree-3 polynomial (coefficients fitted for the
-// smallest relative error on [-1/2, 1/2]: at most 7.5e-5, far below the bf16
-// rounding the result gets next) and 2^n is added to the exponent field.
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-  float x0, x1;
-  unpack2(x2, x0, x1);
-  const uint64_t xc = f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const uint64_t t = fadd2(xc, f32x2(12582912.f, 12582912.f));
-  const uint64_t n = fadd2(t, f32x2(-12582912.f, -12582912.f));
-  const uint64_t f = ffma2(n, f32x2(-1.f, -1.f), xc);
-  uint64_t p = ffma2(f32x2(0.05517132f, 0.05517132f), f, f32x2(0.24261054f, 0.24261054f));
-  p = ffma2(p, f, f32x2(0.69326097f, 0.69326097f));
-  p = ffma2(p, f, f32x2(0.99992812f, 0.99992812f));
-  float t0, t1, p0, p1;
-  unpack2(t, t0, t1);
-  unpack2(p, p0, p1);
-  return f32x2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
-               __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
