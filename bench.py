@@ -376,7 +376,8 @@ def run_gpu(args, rank, world, local_rank):
             "theoretical_speedup_tiles": round(dense_flops / flops, 3)},
         "e2e": {"value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "api": "sparse_attention (pinned host buffers; copies overlap the passes over 8 head groups)"},
+                "api": "sparse_attention -> C-ABI svg_attention_step_host (pinned host buffers; the library's three "
+                       "streams overlap the copies with the passes over 8 head groups)"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }

@@ -252,6 +252,39 @@ svg_status svg_attention_step(const svg_shape* shape, const svg_params* params,
                               int32_t* row_ptr, int32_t* col, uint8_t* full, int64_t capacity,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* The whole step on HOST buffers (the end-to-end call of a caller whose tensors
+ * live in host memory).  The B*H heads are split into `groups` head groups
+ * (sizes differ by at most one): group g+1's Q, K and V are copied to the
+ * device while group g runs the five passes of svg_attention_step, and each
+ * group's output is copied back while the next group runs, on three streams
+ * the library creates once per device.  Every stage is per head, so the
+ * output equals svg_attention_step on the whole problem (head kinds and
+ * attention rows alike).
+ *   q_host, k_host, v_host: host bf16 [B,H,L,d] (model order);
+ *   gamma_q_host, gamma_k_host: host fp32 [d]; sample_idx_host: host int32 [n];
+ *   out_host: host bf16 [B,H,L,d], the output in model order;
+ *   head_kind_out_host: host uint8 [B*H] (the profiled kinds) or NULL;
+ *   1 <= groups <= B*H;
+ *   workspace: device scratch of svg_attention_step_host_workspace_size()
+ *     bytes, 16-byte aligned, owned by the caller: full-size device copies of
+ *     Q, K, V and O plus one head group's intermediates.
+ * The work starts after the caller's earlier work on `stream`, and `stream`
+ * waits for the last copy: synchronise it before reading out_host.  The host
+ * buffers should be pinned (cudaHostAlloc / cudaHostRegister); with pageable
+ * memory the copies still happen but do not overlap the passes.  Calls that
+ * share a workspace must be ordered on the GPU (the same stream, or
+ * synchronised).  The RoPE table is built on the host into a pinned staging
+ * buffer the library keeps per device.  Errors as for svg_attention_step, plus
+ * SVG_ERR_CAPACITY for a workspace below the size required. */
+size_t svg_attention_step_host_workspace_size(const svg_shape* shape, const svg_params* params, int n,
+                                              int groups);
+svg_status svg_attention_step_host(const svg_shape* shape, const svg_params* params,
+                                   const uint16_t* q_host, const uint16_t* k_host, const uint16_t* v_host,
+                                   const float* gamma_q_host, const float* gamma_k_host,
+                                   const int32_t* sample_idx_host, int n, uint16_t* out_host,
+                                   uint8_t* head_kind_out_host, int groups, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* ------------------------------ semantic-aware permutation ("Sparse VideoGen2") */
 /* The second workload ("Sparse VideoGen2" explainer, "A. 语义感知排列" and
  * "B. 基于质心的 Top-p 选择"): per head, the video rows of Q and of K are

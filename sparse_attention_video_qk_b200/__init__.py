@@ -16,7 +16,7 @@ video tokens frame-major and text tokens after them)::
 
 ``SparseAttentionLayer`` adds the denoising schedule (dense for the first
 quarter of the steps, then profiled), and ``sparse_attention`` /
-``HostPipeline`` take pinned host tensors and overlap the copies with the
+``HostStep`` take pinned host tensors and overlap the copies with the
 computation.  Each stage is also callable on its own (``qknorm_rope_layout``,
 ``profile_heads``, ``build_block_index``, ``block_sparse_attn``, ...).
 
@@ -36,7 +36,7 @@ from .api import (DENSE, SPATIAL, TEMPORAL, Problem, StepBuffers, attention_step
                   block_index_capacity, block_sparse_attn, build_block_index, inverse_layout, layout,
                   profile_heads, profile_heads_noalloc, profile_heads_raw_q, profile_workspace_size, qknorm_rope, qknorm_rope_layout, rope_table,
                   sample_queries, sparse_attention, sync_status)
-from .api import STEP_DENSE, STEP_PROFILE, STEP_REUSE, HostPipeline, SparseAttentionLayer, step_policy  # noqa: F401
+from .api import STEP_DENSE, STEP_PROFILE, STEP_REUSE, HostStep, SparseAttentionLayer, step_policy  # noqa: F401
 from .api import AdaSpaLayer, adaspa_block_mass, adaspa_select  # noqa: F401
 from .api import (SVG2Layer, svg2_attention, svg2_block_index, svg2_kmeans, svg2_permutation,  # noqa: F401
                   svg2_permute, svg2_select)
@@ -47,7 +47,7 @@ __all__ = [
     "build_block_index",
     "block_sparse_attn", "inverse_layout", "attention_step", "sparse_attention",
     "sample_queries", "rope_table", "block_index_capacity", "profile_workspace_size", "sync_status",
-    "STEP_DENSE", "STEP_PROFILE", "STEP_REUSE", "step_policy", "SparseAttentionLayer", "HostPipeline",
+    "STEP_DENSE", "STEP_PROFILE", "STEP_REUSE", "step_policy", "SparseAttentionLayer", "HostStep",
     "AdaSpaLayer", "adaspa_block_mass", "adaspa_select",
     "SVG2Layer", "svg2_kmeans", "svg2_permutation", "svg2_select", "svg2_permute", "svg2_block_index",
     "svg2_attention",

@@ -50,6 +50,9 @@ SIGNATURES = {
     "svg_attention_step": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
                                   _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
                                   _vp, _sz, _vp]),
+    "svg_attention_step_host_workspace_size": (_sz, [_SP, _PP, _i32, _i32]),
+    "svg_attention_step_host": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _sz,
+                                       _vp]),
     "svg_sample_queries": (_i32, [ctypes.c_uint64, _i64, _i32, _vp]),
     "svg_adaspa_block_mass": (_i32, [_SP, _PP, _vp, _vp, _vp, _vp, _vp]),
     "svg_adaspa_select": (_i32, [_SP, _PP, _vp, ctypes.c_double, _vp, _vp, _vp, _i64, _vp]),

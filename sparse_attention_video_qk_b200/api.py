@@ -7,7 +7,7 @@ sm_100a kernels.  PyTorch provides device memory and streams.
 from __future__ import annotations
 
 import ctypes
-from dataclasses import dataclass, replace
+from dataclasses import dataclass
 
 import numpy as np
 import torch
@@ -282,97 +282,64 @@ def attention_step(pb: Problem, q, k, v, gamma_q, gamma_k, sample_idx, buffers: 
     return b.out
 
 
-class HostPipeline:
-    """The step on host tensors with the host<->device copies overlapped with
-    the computation.  The B*H heads are split into `chunks` groups: group i+1
-    is copied in (one stream) while group i runs the five passes (a second
-    stream), and each group's output is copied out (a third stream) while the
-    next group runs.  Every stage is per head (profiling scores each head on
-    the shared sample), so the output equals the one-shot step bit for bit.
-    Device inputs and the output are full-size; the step's intermediates are
-    per group and reused."""
+class HostStep:
+    """svg_attention_step_host for one Problem: the step on host tensors, the
+    host<->device copies overlapped with the passes over `groups` head groups
+    inside the library.  Holds the device workspace the call needs (allocated
+    once, reused by every call; calls are ordered on one stream)."""
 
-    def __init__(self, pb: Problem, n_samples: int, chunks: int = 8, device="cuda", sizes=None):
-        bh = pb.B * pb.H
-        if sizes is None:
-            chunks = max(1, min(int(chunks), bh))
-            base, extra = divmod(bh, chunks)
-            sizes = [base + (1 if i < extra else 0) for i in range(chunks)]
-        sizes = [int(n) for n in sizes]
-        if sum(sizes) != bh or min(sizes) < 1:
-            raise ValueError(f"group sizes {sizes} must be positive and sum to B*H = {bh}")
-        self.bounds = []
-        h = 0
-        for n in sizes:
-            self.bounds.append((h, h + n))
-            h += n
-        self.pb, self.bh, self.n = pb, bh, n_samples
-        self.probs = {n: replace(pb, B=1, H=n) for n in {h1 - h0 for h0, h1 in self.bounds}}
-        self.bufs = {n: StepBuffers(p, n_samples, device) for n, p in self.probs.items()}
-        shp = (bh, pb.L, pb.d)
-        self.q, self.k, self.v, self.out = (torch.empty(shp, dtype=torch.bfloat16, device=device) for _ in range(4))
-        self.gq = torch.empty(pb.d, dtype=torch.float32, device=device)
-        self.gk = torch.empty(pb.d, dtype=torch.float32, device=device)
-        self.si = torch.empty(n_samples, dtype=torch.int32, device=device)
-        self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(device=device) for _ in range(3))
+    def __init__(self, pb: Problem, n_samples: int, groups: int = 8, device="cuda"):
+        self.pb, self.n = pb, int(n_samples)
+        self.groups = max(1, min(int(groups), pb.B * pb.H))
+        sh, pr = pb.c_shape(), pb.c_params()
+        size = lib().svg_attention_step_host_workspace_size(ctypes.byref(sh), ctypes.byref(pr), self.n, self.groups)
+        if size == 0:
+            raise ValueError("svg_attention_step_host_workspace_size: invalid shape, parameters or group count")
+        self.workspace = torch.empty(size, dtype=torch.uint8, device=device)
 
-    def __call__(self, q_host, k_host, v_host, gamma_q, gamma_k, sample_idx, out_host=None):
-        pb, bh = self.pb, self.bh
+    def __call__(self, q_host, k_host, v_host, gamma_q, gamma_k, sample_idx, out_host=None, kinds_out=None,
+                 stream=None):
+        """q/k/v_host: bf16 [B,H,L,d] on the host (pinned for overlap); gamma: fp32 [d];
+        sample_idx: int32 [n] (host tensors).  Returns out_host (bf16 [B,H,L,d], pinned
+        if allocated here); kinds_out, if given, receives the uint8 [B*H] head kinds.
+        The current stream (or `stream`) waits for the last copy."""
+        pb = self.pb
         if out_host is None:
             out_host = torch.empty(q_host.shape, dtype=torch.bfloat16, pin_memory=True)
-        flat = lambda t: t.reshape(bh, pb.L, pb.d)
-        qh, kh, vh, oh = flat(q_host), flat(k_host), flat(v_host), flat(out_host)
-        caller = torch.cuda.current_stream()
-        # inputs are overwritten only after the previous call's passes are done
-        self.s_in.wait_stream(caller)
-        self.s_in.wait_stream(self.s_comp)
-        ev_in = []
-        with torch.cuda.stream(self.s_in):
-            self.gq.copy_(gamma_q, non_blocking=True)
-            self.gk.copy_(gamma_k, non_blocking=True)
-            self.si.copy_(sample_idx, non_blocking=True)
-            for h0, h1 in self.bounds:
-                self.q[h0:h1].copy_(qh[h0:h1], non_blocking=True)
-                self.k[h0:h1].copy_(kh[h0:h1], non_blocking=True)
-                self.v[h0:h1].copy_(vh[h0:h1], non_blocking=True)
-                ev = torch.cuda.Event()
-                ev.record(self.s_in)
-                ev_in.append(ev)
-        # the output rows of a group are read back only after its passes
-        self.s_out.wait_stream(caller)
-        for (h0, h1), ev in zip(self.bounds, ev_in):
-            n = h1 - h0
-            b = self.bufs[n]
-            self.s_comp.wait_event(ev)
-            b.out = self.out[h0:h1]
-            attention_step(self.probs[n], self.q[h0:h1], self.k[h0:h1], self.v[h0:h1], self.gq, self.gk, self.si,
-                           b, stream=self.s_comp)
-            done = torch.cuda.Event()
-            done.record(self.s_comp)
-            self.s_out.wait_event(done)
-            with torch.cuda.stream(self.s_out):
-                oh[h0:h1].copy_(self.out[h0:h1], non_blocking=True)
-        caller.wait_stream(self.s_out)
+        for t in (q_host, k_host, v_host, gamma_q, gamma_k, sample_idx, out_host):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError("host tensors must be contiguous CPU tensors")
+        gq = gamma_q.to(torch.float32).contiguous()
+        gk = gamma_k.to(torch.float32).contiguous()
+        si = sample_idx.to(torch.int32).contiguous()
+        if int(si.numel()) != self.n:
+            raise ValueError(f"{si.numel()} sampled rows; this HostStep was made for {self.n}")
+        sh, pr = pb.c_shape(), pb.c_params()
+        cs = torch.cuda.current_stream(self.workspace.device) if stream is None else stream
+        check(lib().svg_attention_step_host(ctypes.byref(sh), ctypes.byref(pr), _p(q_host), _p(k_host), _p(v_host),
+                                            _p(gq), _p(gk), _p(si), self.n, _p(out_host), _p(kinds_out), self.groups,
+                                            _p(self.workspace), self.workspace.numel(), _stream(cs)),
+              "svg_attention_step_host")
         return out_host
 
 
-_PIPELINES = {}
+_HOST_STEPS = {}
 
 
 def sparse_attention(pb: Problem, q_host, k_host, v_host, gamma_q, gamma_k, sample_idx, out_host=None,
-                     device="cuda", chunks: int = 8, pipeline: HostPipeline = None):
+                     device="cuda", groups: int = 8, host_step: HostStep = None):
     """End-to-end call on host tensors: Q/K/V (bf16 [B,H,L,d], pinned so the
     copies are asynchronous), gamma and the sample go in, O comes back in
-    `out_host` (allocated pinned if None).  The copies overlap the passes
-    through a HostPipeline of `chunks` head groups (created once per shape and
-    cached, or passed in).  Work is ordered after the current stream, and the
-    current stream waits for the last copy.  Returns out_host."""
-    if pipeline is None:
-        key = (pb, int(sample_idx.numel()), int(chunks), str(device))
-        pipeline = _PIPELINES.get(key)
-        if pipeline is None:
-            pipeline = _PIPELINES[key] = HostPipeline(pb, int(sample_idx.numel()), chunks, device)
-    return pipeline(q_host, k_host, v_host, gamma_q, gamma_k, sample_idx, out_host)
+    `out_host` (allocated pinned if None), through svg_attention_step_host with
+    `groups` head groups (its workspace created once per shape and cached, or
+    passed in as `host_step`).  Work is ordered after the current stream, and
+    the current stream waits for the last copy.  Returns out_host."""
+    if host_step is None:
+        key = (pb, int(sample_idx.numel()), int(groups), str(device))
+        host_step = _HOST_STEPS.get(key)
+        if host_step is None:
+            host_step = _HOST_STEPS[key] = HostStep(pb, int(sample_idx.numel()), groups, device)
+    return host_step(q_host, k_host, v_host, gamma_q, gamma_k, sample_idx, out_host)
 
 
 # ------------------------------------------- semantic-aware permutation --

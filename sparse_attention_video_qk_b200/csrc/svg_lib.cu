@@ -824,3 +824,5 @@ svg_status svg_adaspa_select(const svg_shape* s, const svg_params* p, const floa
 
 // Profiling with library-owned scratch (svg_profile_heads_noalloc).
 #include "profile_noalloc.cuh"
+// The step on host buffers, copies overlapped with the passes (svg_attention_step_host).
+#include "host_step.cuh"

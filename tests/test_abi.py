@@ -165,6 +165,27 @@ def test_svg2_attention_rejects_null_pointers(L):
     assert e.value.status == C.SVG_ERR_INVALID_ARG
 
 
+def test_host_step_argument_errors(L):
+    """svg_attention_step_host rejects bad group counts and a short workspace
+    before any CUDA call; the workspace size grows with nothing but the shape."""
+    wl = W.TINY
+    pb = api.Problem.from_workload(wl)
+    sh, pr = pb.c_shape(), pb.c_params()
+    p = ctypes.c_void_p(256)
+    size = L.svg_attention_step_host_workspace_size(ctypes.byref(sh), ctypes.byref(pr), 16, 1)
+    assert size >= 4 * wl.B * wl.H * wl.L * wl.d * 2
+    assert L.svg_attention_step_host_workspace_size(ctypes.byref(sh), ctypes.byref(pr), 16, 0) == 0
+    assert L.svg_attention_step_host_workspace_size(ctypes.byref(sh), ctypes.byref(pr), 16, wl.B * wl.H + 1) == 0
+    call = lambda groups, ws_bytes, n=16: L.svg_attention_step_host(
+        ctypes.byref(sh), ctypes.byref(pr), p, p, p, p, p, p, n, p, None, groups, p, ws_bytes, None)
+    assert call(0, size) == C.SVG_ERR_INVALID_ARG
+    assert call(wl.B * wl.H + 1, size) == C.SVG_ERR_INVALID_ARG
+    assert call(1, size, n=0) == C.SVG_ERR_INVALID_ARG
+    assert call(1, size - 1) == C.SVG_ERR_CAPACITY
+    assert L.svg_attention_step_host(ctypes.byref(sh), ctypes.byref(pr), p, p, p, p, p, p, 16, p, None, 1,
+                                     ctypes.c_void_p(8), size, None) == C.SVG_ERR_ALIGNMENT
+
+
 def test_noalloc_capacity_limit(L):
     """The no-alloc profiling entry rejects shapes whose one key chunk of
     partials does not fit its 16 MiB scratch, before any CUDA call."""

@@ -361,19 +361,21 @@ def test_full_step_end_to_end(key, head_layout_out):
     assert_attention_close(host_bits(out).reshape(-1, wl.d)[rows], ref, MAX_ABS, MEAN_ABS, key)
 
 
-@pytest.mark.parametrize("key,chunks", [("wan", 4), ("wan", 5), ("batch2", 3), ("tiny", 1), ("batch2", [1, 2, 1])])
-def test_host_pipeline_chunks_match_one_shot_step(key, chunks):
-    """Head groups copied in, computed and copied out on three streams give
-    the one-shot device step's bits, for even and uneven groups and B > 1."""
+@pytest.mark.parametrize("key,groups", [("wan", 4), ("wan", 5), ("batch2", 3), ("tiny", 1), ("batch2", 4)])
+def test_host_step_groups_match_one_shot_step(key, groups):
+    """svg_attention_step_host (head groups copied in, computed and copied out
+    on the library's three streams) gives the one-shot device step's bits and
+    head kinds, for even and uneven groups, one head per group and B > 1, on
+    two calls in a row (the second reuses the workspace)."""
     wl, inp, _, _ = case(key)
     pb = pb_of(wl)
     pin = lambda a: torch.from_numpy(a).view(torch.bfloat16).pin_memory()
-    pipe = (svg.HostPipeline(pb, wl.n_samples, sizes=chunks) if isinstance(chunks, list)
-            else svg.HostPipeline(pb, wl.n_samples, chunks=chunks))
+    step = svg.HostStep(pb, wl.n_samples, groups=groups)
     args = (pin(inp["q"]), pin(inp["k"]), pin(inp["v"]), torch.from_numpy(inp["gamma_q"]).pin_memory(),
             torch.from_numpy(inp["gamma_k"]).pin_memory(), torch.from_numpy(inp["sample_idx"]).pin_memory())
-    out_h = pipe(*args)
-    out_h2 = pipe(*args)          # a second call reuses every buffer
+    kinds_h = torch.empty(wl.B * wl.H, dtype=torch.uint8).pin_memory()
+    out_h = step(*args, kinds_out=kinds_h)
+    out_h2 = step(*args)
     torch.cuda.synchronize()
     buf = svg.StepBuffers(pb, wl.n_samples)
     out_d = svg.attention_step(pb, *(dev(inp[k]) for k in ("q", "k", "v", "gamma_q", "gamma_k", "sample_idx")), buf)
@@ -381,6 +383,7 @@ def test_host_pipeline_chunks_match_one_shot_step(key, chunks):
     ref = out_d.cpu().view(torch.int16)
     assert torch.equal(out_h.view(torch.int16), ref)
     assert torch.equal(out_h2.view(torch.int16), ref)
+    assert torch.equal(kinds_h, buf.kinds.cpu())
 
 
 def test_host_buffer_api_matches_device_api():
