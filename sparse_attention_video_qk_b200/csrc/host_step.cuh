@@ -48,13 +48,10 @@ inline bool layout_of(const svg_shape* s, const svg_params* p, int n, int groups
   const svg_shape gs = group_shape(s, gmax);
   L->capacity = svg_block_index_capacity(&gs, p);
   if (L->capacity <= 0) return false;
-  // the profiling scratch depends on the head count (key chunks per head)
-  L->prof_bytes = 0;
-  for (int g = 0; g < groups && g < 2 + BH % groups; g++) {
-    const svg_shape gg = group_shape(s, group_size(BH, groups, g));
-    L->prof_bytes = std::max(L->prof_bytes, svg_profile_workspace_size(&gg, n));
-  }
-  L->prof_bytes = std::max(L->prof_bytes, svg_profile_workspace_size(&gs, n));
+  // the profiling scratch depends on the head count (key chunks per head):
+  // the larger of the two group sizes' needs
+  const svg_shape gsmall = group_shape(s, BH / groups);
+  L->prof_bytes = std::max(svg_profile_workspace_size(&gs, n), svg_profile_workspace_size(&gsmall, n));
   L->table_floats = svg_rope_table_size(s, p);
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -142,6 +139,7 @@ extern "C" svg_status svg_attention_step_host(const svg_shape* s, const svg_para
                                               const int32_t* sample_idx_host, int n, uint16_t* out_host,
                                               uint8_t* head_kind_out_host, int groups, void* workspace,
                                               size_t workspace_bytes, void* stream) {
+  svg::NvtxRange nvtx_range_("svg_attention_step_host");
   using namespace svg;
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;

@@ -42,6 +42,7 @@ inline svg_status noalloc_scratch(float** out) {
 extern "C" svg_status svg_profile_heads_noalloc(const svg_shape* s, const svg_params* p, const uint16_t* qn,
                                                 const uint16_t* kn, const uint16_t* v, const int32_t* sample_idx,
                                                 int n, float* mse_out, uint8_t* head_kind_out, void* stream) {
+  svg::NvtxRange nvtx_range_("svg_profile_heads_noalloc");
   using namespace svg;
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;

@@ -8,9 +8,21 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "svg.h"
 
 namespace svg {
+
+// A named NVTX range over one C-ABI call (host side), so a profiler timeline
+// shows each call's span and the kernels it launched.  Costs a pointer test
+// when no tool is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Error word codes (device side).  Written with atomicOr, read and cleared by
 // svg_sync_status().

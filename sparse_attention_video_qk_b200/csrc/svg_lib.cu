@@ -371,6 +371,7 @@ svg_status svg_qknorm_rope_layout(const svg_shape* s, const svg_params* p, int f
                                   const uint16_t* k, const uint16_t* v, const float* gamma_q, const float* gamma_k,
                                   const float* rope_table, const uint8_t* head_kind, uint16_t* q_out,
                                   uint16_t* k_out, uint16_t* v_out, void* stream) {
+  svg::NvtxRange nvtx_range_("svg_qknorm_rope_layout");
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if (!p) return SVG_ERR_INVALID_ARG;
@@ -417,6 +418,7 @@ svg_status svg_qknorm_rope_layout(const svg_shape* s, const svg_params* p, int f
 
 svg_status svg_inverse_layout(const svg_shape* s, const uint8_t* head_kind, const uint16_t* src, uint16_t* dst,
                               void* stream) {
+  svg::NvtxRange nvtx_range_("svg_inverse_layout");
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if (!head_kind || !src || !dst || src == dst) return SVG_ERR_INVALID_ARG;
@@ -436,6 +438,7 @@ svg_status svg_inverse_layout(const svg_shape* s, const uint8_t* head_kind, cons
 svg_status svg_profile_heads(const svg_shape* s, const svg_params* p, const uint16_t* qn, const uint16_t* kn,
                              const uint16_t* v, const int32_t* sample_idx, int n, void* workspace,
                              size_t workspace_bytes, float* mse_out, uint8_t* head_kind_out, void* stream) {
+  svg::NvtxRange nvtx_range_("svg_profile_heads");
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if ((st = check_params(s, p, false)) != SVG_OK) return st;
@@ -453,6 +456,7 @@ svg_status svg_profile_heads_raw_q(const svg_shape* s, const svg_params* p, cons
                                    const float* rope_table, const uint16_t* kn, const uint16_t* v,
                                    const int32_t* sample_idx, int n, void* workspace, size_t workspace_bytes,
                                    float* mse_out, uint8_t* head_kind_out, void* stream) {
+  svg::NvtxRange nvtx_range_("svg_profile_heads_raw_q");
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if ((st = check_params(s, p, false)) != SVG_OK) return st;
@@ -470,6 +474,7 @@ svg_status svg_profile_heads_raw_q(const svg_shape* s, const svg_params* p, cons
 
 svg_status svg_build_block_index(const svg_shape* s, const svg_params* p, const uint8_t* head_kind,
                                  int32_t* row_ptr, int32_t* col, uint8_t* full, int64_t capacity, void* stream) {
+  svg::NvtxRange nvtx_range_("svg_build_block_index");
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if ((st = check_params(s, p, true)) != SVG_OK) return st;
@@ -558,6 +563,7 @@ svg_status svg_block_sparse_attn(const svg_shape* s, const svg_params* p, const 
                                  const uint16_t* v, const uint8_t* head_kind, const int32_t* row_ptr,
                                  const int32_t* col, const uint8_t* full, uint16_t* out, float* lse_out,
                                  void* stream) {
+  svg::NvtxRange nvtx_range_("svg_block_sparse_attn");
   return attention_launch(s, p, q, k, v, head_kind, row_ptr, col, full, out, lse_out, 0, stream);
 }
 
@@ -565,6 +571,7 @@ svg_status svg_block_sparse_attn_model_order(const svg_shape* s, const svg_param
                                              const uint16_t* k, const uint16_t* v, const uint8_t* head_kind,
                                              const int32_t* row_ptr, const int32_t* col, const uint8_t* full,
                                              uint16_t* out, float* lse_out, void* stream) {
+  svg::NvtxRange nvtx_range_("svg_block_sparse_attn_model_order");
   return attention_launch(s, p, q, k, v, head_kind, row_ptr, col, full, out, lse_out, 1, stream);
 }
 
@@ -574,6 +581,7 @@ svg_status svg_attention_step(const svg_shape* s, const svg_params* p, const uin
                               uint16_t* qp, uint16_t* kp, uint16_t* vp, uint16_t* op, uint16_t* out,
                               uint8_t* head_kind_out, float* mse_out, int32_t* row_ptr, int32_t* col, uint8_t* full,
                               int64_t capacity, void* workspace, size_t workspace_bytes, void* stream) {
+  svg::NvtxRange nvtx_range_("svg_attention_step");
   svg_status st;
   if (!head_kind_out) return SVG_ERR_INVALID_ARG;
   // 1. QK-Norm + RoPE of K (profiling reads every normalised key)
@@ -611,6 +619,7 @@ size_t svg2_kmeans_workspace_size(const svg_shape* s, int C) {
 
 svg_status svg2_kmeans(const svg_shape* s, const uint16_t* x, int C, int iters, int init, float* cent,
                        uint8_t* assign, int32_t* counts, void* workspace, size_t workspace_bytes, void* stream) {
+  svg::NvtxRange nvtx_range_("svg2_kmeans");
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   const int Lv = s->F * s->Hs * s->Ws;
@@ -653,6 +662,7 @@ svg_status svg2_kmeans(const svg_shape* s, const uint16_t* x, int C, int iters, 
 
 svg_status svg2_permutation(const svg_shape* s, const uint8_t* assign, int C, int32_t* perm, int32_t* off,
                             void* stream) {
+  svg::NvtxRange nvtx_range_("svg2_permutation");
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if (!assign || !perm || !off || C < 1 || C > kMaxClusters) return SVG_ERR_INVALID_ARG;
@@ -663,6 +673,7 @@ svg_status svg2_permutation(const svg_shape* s, const uint8_t* assign, int C, in
 
 svg_status svg2_select(const svg_shape* s, const svg_params* p, const float* cq, const float* ck,
                        const int32_t* counts_k, int Cq, int Ck, double top_p, uint64_t* sel, void* stream) {
+  svg::NvtxRange nvtx_range_("svg2_select");
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if ((st = check_params(s, p, false)) != SVG_OK) return st;
@@ -678,6 +689,7 @@ svg_status svg2_select(const svg_shape* s, const svg_params* p, const float* cq,
 svg_status svg2_permute(const svg_shape* s, const int32_t* perm_q, const int32_t* perm_k, const uint16_t* q,
                         const uint16_t* k, const uint16_t* v, uint16_t* q_out, uint16_t* k_out, uint16_t* v_out,
                         void* stream) {
+  svg::NvtxRange nvtx_range_("svg2_permute");
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if (!perm_q || !perm_k || !q || !k || !v || !q_out || !k_out || !v_out) return SVG_ERR_INVALID_ARG;
@@ -711,6 +723,7 @@ svg_status svg2_permute(const svg_shape* s, const int32_t* perm_q, const int32_t
 svg_status svg2_build_block_index(const svg_shape* s, const svg_params* p, int Cq, int Ck, const int32_t* qoff,
                                   const int32_t* koff, const uint64_t* sel, int32_t* row_ptr, int32_t* col,
                                   uint8_t* full, int64_t capacity, void* stream) {
+  svg::NvtxRange nvtx_range_("svg2_build_block_index");
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if ((st = check_params(s, p, true)) != SVG_OK) return st;
@@ -745,6 +758,7 @@ svg_status svg2_attention(const svg_shape* s, const svg_params* p, const uint16_
                           const uint16_t* v, int Cq, int Ck, const int32_t* qoff, const int32_t* koff,
                           const uint64_t* sel, const int32_t* perm_q, const int32_t* row_ptr, const int32_t* col,
                           const uint8_t* full, uint16_t* out, float* lse_out, void* stream) {
+  svg::NvtxRange nvtx_range_("svg2_attention");
   if (!qoff || !koff || !sel || !perm_q) return SVG_ERR_INVALID_ARG;
   if (Cq < 1 || Cq > kMaxClusters || Ck < 1 || Ck > kMaxClusters) return SVG_ERR_INVALID_ARG;
   AttnArgs c{};
@@ -761,6 +775,7 @@ svg_status svg2_attention(const svg_shape* s, const svg_params* p, const uint16_
 
 svg_status svg_adaspa_block_mass(const svg_shape* s, const svg_params* p, const uint16_t* q, const uint16_t* k,
                                  const float* lse, float* mass, void* stream) {
+  svg::NvtxRange nvtx_range_("svg_adaspa_block_mass");
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if ((st = check_params(s, p, true)) != SVG_OK) return st;
@@ -790,6 +805,7 @@ svg_status svg_adaspa_block_mass(const svg_shape* s, const svg_params* p, const 
 
 svg_status svg_adaspa_select(const svg_shape* s, const svg_params* p, const float* mass, double top_p,
                              int32_t* row_ptr, int32_t* col, uint8_t* full, int64_t capacity, void* stream) {
+  svg::NvtxRange nvtx_range_("svg_adaspa_select");
   svg_status st = check_shape(s);
   if (st != SVG_OK) return st;
   if ((st = check_params(s, p, true)) != SVG_OK) return st;
