@@ -27,7 +27,7 @@ inline int group_start(int BH, int groups, int g) { return g * (BH / groups) + (
 
 // Byte offsets of the workspace's buffers.
 struct Layout {
-  size_t q, k, v, out, kinds, mse, gamma_q, gamma_k, sample, table;  // whole problem
+  size_t q, k, v, out, kinds, gamma_q, gamma_k, sample, table;  // whole problem
   size_t kn, qp, kp, vp, row_ptr, col, full, prof;                    // one head group (the largest)
   size_t total;
   int64_t capacity;
@@ -64,7 +64,6 @@ inline bool layout_of(const svg_shape* s, const svg_params* p, int n, int groups
   L->v = take(BH * head_bytes);
   L->out = take(BH * head_bytes);
   L->kinds = take(static_cast<size_t>(BH));
-  L->mse = take(static_cast<size_t>(BH) * 2 * sizeof(float));
   L->gamma_q = take(static_cast<size_t>(s->d) * sizeof(float));
   L->gamma_k = take(static_cast<size_t>(s->d) * sizeof(float));
   L->sample = take(static_cast<size_t>(n) * sizeof(int32_t));
@@ -165,7 +164,6 @@ extern "C" svg_status svg_attention_step_host(const svg_shape* s, const svg_para
   uint16_t* v = reinterpret_cast<uint16_t*>(at(L.v));
   uint16_t* out = reinterpret_cast<uint16_t*>(at(L.out));
   uint8_t* kinds = at(L.kinds);
-  float* mse = reinterpret_cast<float*>(at(L.mse));
   float* gq = reinterpret_cast<float*>(at(L.gamma_q));
   float* gk = reinterpret_cast<float*>(at(L.gamma_k));
   int32_t* sample = reinterpret_cast<int32_t*>(at(L.sample));
@@ -227,7 +225,7 @@ extern "C" svg_status svg_attention_step_host(const svg_shape* s, const svg_para
     st = svg_attention_step(&gs, p, q + off, k + off, v + off, gq, gk, table, sample, n, nullptr,
                             reinterpret_cast<uint16_t*>(at(L.kn)), reinterpret_cast<uint16_t*>(at(L.qp)),
                             reinterpret_cast<uint16_t*>(at(L.kp)), reinterpret_cast<uint16_t*>(at(L.vp)), nullptr,
-                            out + off, kinds + h0, mse + 2 * static_cast<size_t>(h0),
+                            out + off, kinds + h0, nullptr,
                             reinterpret_cast<int32_t*>(at(L.row_ptr)), reinterpret_cast<int32_t*>(at(L.col)),
                             at(L.full), L.capacity, at(L.prof), L.prof_bytes, ds->comp);
     if (st != SVG_OK) return st;
