@@ -682,8 +682,9 @@ def run_sweep(args):
             "steps_per_point": args.steps, "warmup": args.warmup, "statistic": "median CUDA-event ms",
             "dense": {"ms": round(dense_ms, 3), "tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 1),
                       "tflop": round(dense_flops / 1e12, 3)},
-            "peak_bf16_sustained": pk["bf16_tflops_sustained"], "peak_source": pk_src,
-            "points": points, "clocks": clk.summary(),
+            "peak_bf16_burst": pk["bf16_tflops"], "peak_source": pk_src,
+            "points": [dict(p, frac_of_burst_peak=round(p["tflops"] / pk["bf16_tflops"], 4)) for p in points],
+            "clocks": clk.summary(),
             "data": "synthetic N(0,1) bf16 Q/K/V, head kinds forced"}
 
 
