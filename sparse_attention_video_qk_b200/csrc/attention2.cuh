@@ -18,11 +18,13 @@
 //     P.V and S.  The commit behind S_w(j) covers P.V_w(j-1), so a query tile's
 //     O accumulator is idle whenever its softmax holds S: rescales need no wait;
 //   * the softmax reads S once per tile in 32-column chunks: it exponentiates
-//     with the running maximum while it tracks the tile's own, keeps the packed
-//     P row (64 registers) and stores it only once the tile maximum is known
-//     not to outgrow the running one by more than 2^8; otherwise (and on the
-//     first tile) it rescales O and recomputes P from S, still in TMEM.  It
-//     fetches the next tile's list entries one tile ahead.
+//     against the running maximum without tracking the tile's own, keeps the
+//     packed P row (64 registers) and stores it once every row sum of the tile
+//     is known to stay below 2^64 (then nothing can overflow, however far the
+//     running maximum lags).  Otherwise, on the first tile and while a row has
+//     no running maximum yet, it takes the tile's maximum, rescales O and
+//     computes P from S, still in TMEM.  It fetches the next tile's list
+//     entries one tile ahead.
 // Every mbarrier wait is bounded; on time-out the kernel records
 // kErrTimeout, drains its outstanding copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -379,13 +381,14 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
             for (int c = 0; c < 32; c++)
               if (!((keep >> c) & 1u)) v[c] = __float_as_uint(-INFINITY);
           } else {
+            // kept columns: the row's window [lo, hi) and the text keys [Lv, Lv + T),
+            // as one 32-bit word (a few instructions instead of two compares per column)
+            const int a0 = min(max(lo - k0, 0), 32), a1 = min(max(hi - k0, 0), 32);
+            const int t0 = min(max(g.Lv - k0, 0), 32), t1 = min(max(g.Lv + g.T - k0, 0), 32);
+            const uint32_t keep = (a0 < a1 ? span_bits(a0, a1) : 0u) | (t0 < t1 ? span_bits(t0, t1) : 0u);
 #pragma unroll
-            for (int c = 0; c < 32; c++) {
-              const int kk = k0 + c;
-              const bool keep = (static_cast<unsigned>(kk - lo) < static_cast<unsigned>(hi - lo)) ||
-                                (static_cast<unsigned>(kk - g.Lv) < static_cast<unsigned>(g.T));
-              if (!keep) v[c] = __float_as_uint(-INFINITY);
-            }
+            for (int c = 0; c < 32; c++)
+              if (!((keep >> c) & 1u)) v[c] = __float_as_uint(-INFINITY);
           }
         }
       };
@@ -437,7 +440,7 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
           body(v, q);
         }
       };
-      bool rescale = (j == 0);
+      bool rescale;
       if (j > 0 && __all_sync(0xffffffffu, m_use != -INFINITY)) {
         // Every row has a running maximum: exponentiate against it without tracking
         // the tile's maximum.  The result stands while the tile's row sum of
@@ -452,20 +455,14 @@ __global__ void __launch_bounds__(Attn2Cfg<D>::THREADS, 1)
         unpack2(acc[1], s2, s3);
         rescale = __any_sync(0xffffffffu, !(((s0 + s1) + (s2 + s3)) < 0x1p64f));
         if (rescale) pass([&](const uint32_t* v, int q) { chunk_max(v, m8); });
-      } else if (j > 0) {
-        // some row has seen no kept key yet: exponentiate and track the maximum;
-        // the result stands unless it outgrows the running one by 2^8
-        const float msub = (m_use == -INFINITY) ? 0.f : m_use;
-        const uint64_t nm2 = f32x2(-msub, -msub);
-        pass([&](const uint32_t* v, int q) {
-          chunk_max(v, m8);
-          chunk_exp(v, pk + 16 * q, acc, nm2);
-        });
-        const float mxs = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
-        rescale = __any_sync(0xffffffffu, mxs > m_use + 8.0f);
       } else {
-        // first tile: the running maximum starts at the tile's own
+        // First tile, or a row of the warp has seen no kept key yet: the tile's
+        // maximum first, then P against it.  (A combined max-and-exponentiate pass
+        // for the second case was measured slower: the kernel's code grew by a
+        // third, and sparse lists, which meet this case often, ran up to 18%
+        // slower.)
         pass([&](const uint32_t* v, int q) { chunk_max(v, m8); });
+        rescale = true;
       }
       if (rescale) {
         const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
