@@ -432,6 +432,25 @@ int64_t svg_block_index_capacity(const svg_shape* shape, const svg_params* param
 /* Device scratch bytes svg_profile_heads needs for n sampled rows. */
 size_t svg_profile_workspace_size(const svg_shape* shape, int n);
 
+/* Device scratch bytes that every entry point taking a caller workspace needs
+ * for this shape and parameters: svg_profile_heads and svg_profile_heads_raw_q
+ * with any n from 1 to 64 (the scratch does not grow with n).  0 for a null
+ * pointer, a shape the library rejects, negative window parameters, or tiles
+ * other than block_k = 64 and block_q in {64, 128}. */
+size_t svg_workspace_size(const svg_shape* shape, const svg_params* params);
+
+/* Releases the library's cached state: on every device that has run
+ * svg_attention_step_host, it waits for the library's own three streams to
+ * finish, then destroys them and their events and frees the pinned staging
+ * buffer of the RoPE table.  Nothing else is cached (the fixed scratch of
+ * svg_profile_heads_noalloc is a device array that lives as long as the
+ * library).  The next svg_attention_step_host creates them again.  Call it
+ * from one thread, with no call of the library in flight on another.
+ * Restores the calling thread's current device.  Returns SVG_OK, or
+ * SVG_ERR_CUDA if a synchronisation or a release failed (the state is
+ * dropped all the same).  Touches no GPU when nothing is cached. */
+svg_status svg_release(void);
+
 /* Synchronises `stream`, then reads and clears this device's error word:
  * SVG_OK, SVG_ERR_TIMEOUT or SVG_ERR_CAPACITY (or SVG_ERR_CUDA if the
  * synchronisation itself failed). */

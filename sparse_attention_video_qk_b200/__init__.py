@@ -34,8 +34,9 @@ Q and K (``qknorm_rope``)::
 from ._lib import SVGError, lib  # noqa: F401
 from .api import (DENSE, SPATIAL, TEMPORAL, Problem, StepBuffers, attention_step,  # noqa: F401
                   block_index_capacity, block_sparse_attn, build_block_index, inverse_layout, layout,
-                  profile_heads, profile_heads_noalloc, profile_heads_raw_q, profile_workspace_size, qknorm_rope, qknorm_rope_layout, rope_table,
-                  sample_queries, sparse_attention, sync_status)
+                  profile_heads, profile_heads_noalloc, profile_heads_raw_q, profile_workspace_size, qknorm_rope,
+                  qknorm_rope_layout, release, rope_table, sample_queries, sparse_attention, sync_status,
+                  workspace_size)
 from .api import STEP_DENSE, STEP_PROFILE, STEP_REUSE, HostStep, SparseAttentionLayer, step_policy  # noqa: F401
 from .api import AdaSpaLayer, adaspa_block_mass, adaspa_select  # noqa: F401
 from .api import (SVG2Layer, svg2_attention, svg2_block_index, svg2_kmeans, svg2_permutation,  # noqa: F401
@@ -46,7 +47,8 @@ __all__ = [
     "qknorm_rope", "qknorm_rope_layout", "layout", "profile_heads", "profile_heads_noalloc", "profile_heads_raw_q",
     "build_block_index",
     "block_sparse_attn", "inverse_layout", "attention_step", "sparse_attention",
-    "sample_queries", "rope_table", "block_index_capacity", "profile_workspace_size", "sync_status",
+    "sample_queries", "rope_table", "block_index_capacity", "profile_workspace_size", "workspace_size", "release",
+    "sync_status",
     "STEP_DENSE", "STEP_PROFILE", "STEP_REUSE", "step_policy", "SparseAttentionLayer", "HostStep",
     "AdaSpaLayer", "adaspa_block_mass", "adaspa_select",
     "SVG2Layer", "svg2_kmeans", "svg2_permutation", "svg2_select", "svg2_permute", "svg2_block_index",

@@ -69,6 +69,8 @@ SIGNATURES = {
     "svg_rope_table_fill": (_i32, [_SP, _PP, _vp]),
     "svg_block_index_capacity": (_i64, [_SP, _PP]),
     "svg_profile_workspace_size": (_sz, [_SP, _i32]),
+    "svg_workspace_size": (_sz, [_SP, _PP]),
+    "svg_release": (_i32, []),
     "svg_sync_status": (_i32, [_vp]),
     "svg_selftest_wait_timeout": (_i32, [_vp]),
     "svg_status_string": (ctypes.c_char_p, [_i32]),

@@ -113,6 +113,20 @@ def profile_workspace_size(pb: Problem, n: int) -> int:
     return int(lib().svg_profile_workspace_size(ctypes.byref(sh), n))
 
 
+def workspace_size(pb: Problem) -> int:
+    """svg_workspace_size: device scratch bytes of the workspace-taking calls."""
+    sh, pr = pb.c_shape(), pb.c_params()
+    return int(lib().svg_workspace_size(ctypes.byref(sh), ctypes.byref(pr)))
+
+
+def release():
+    """svg_release: waits for and frees the library's cached streams, events and
+    pinned staging (the host-buffer step's).  Also drops this module's cached
+    HostStep workspaces."""
+    _HOST_STEPS.clear()
+    check(lib().svg_release(), "svg_release")
+
+
 def sync_status(stream=None):
     """Synchronise the stream and raise if a kernel reported an error."""
     check(lib().svg_sync_status(_stream(stream)), "svg_sync_status")

@@ -118,8 +118,48 @@ inline bool ensure(DeviceStreams* ds, size_t need) {
   return true;
 }
 
+// Waits for one device's library streams, then frees its streams, events and
+// pinned staging.  Called with ds->mu held.
+inline bool release(DeviceStreams* ds, int dev) {
+  if (!ds->ready && ds->events.empty() && ds->table_stage == nullptr) return true;
+  bool good = cudaSetDevice(dev) == cudaSuccess;
+  for (cudaStream_t st : {ds->in, ds->comp, ds->out})
+    if (st) good &= cudaStreamSynchronize(st) == cudaSuccess;
+  for (cudaEvent_t e : ds->events) good &= cudaEventDestroy(e) == cudaSuccess;
+  ds->events.clear();
+  if (ds->table_copied) good &= cudaEventDestroy(ds->table_copied) == cudaSuccess;
+  for (cudaStream_t st : {ds->in, ds->comp, ds->out})
+    if (st) good &= cudaStreamDestroy(st) == cudaSuccess;
+  if (ds->table_stage) good &= cudaFreeHost(ds->table_stage) == cudaSuccess;
+  ds->in = ds->comp = ds->out = nullptr;
+  ds->table_copied = nullptr;
+  ds->table_stage = nullptr;
+  ds->table_stage_floats = 0;
+  ds->table_pending = false;
+  ds->ready = false;
+  return good;
+}
+
 }  // namespace hoststep
 }  // namespace svg
+
+extern "C" svg_status svg_release(void) {
+  using namespace svg;
+  int prev = -1;
+  bool touched = false, good = true;
+  for (int dev = 0; dev < hoststep::kMaxDevices; dev++) {
+    hoststep::DeviceStreams* ds = hoststep::device_streams(dev);
+    std::lock_guard<std::mutex> lock(ds->mu);
+    if (!ds->ready && ds->events.empty() && ds->table_stage == nullptr) continue;
+    if (!touched) {
+      touched = true;
+      good &= cudaGetDevice(&prev) == cudaSuccess;
+    }
+    good &= hoststep::release(ds, dev);
+  }
+  if (touched && prev >= 0) good &= cudaSetDevice(prev) == cudaSuccess;
+  return good ? SVG_OK : SVG_ERR_CUDA;
+}
 
 extern "C" size_t svg_attention_step_host_workspace_size(const svg_shape* s, const svg_params* p, int n,
                                                           int groups) {

@@ -350,6 +350,11 @@ size_t svg_profile_workspace_size(const svg_shape* s, int n) {
   return prof_workspace_bytes(BH, s->L, s->d, prof_chunks(BH, s->L));
 }
 
+size_t svg_workspace_size(const svg_shape* s, const svg_params* p) {
+  if (check_shape(s) != SVG_OK || check_params(s, p, true) != SVG_OK) return 0;
+  return svg_profile_workspace_size(s, kProfRows);
+}
+
 svg_status svg_selftest_wait_timeout(void* stream) {
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
   return launch_status();

@@ -106,6 +106,28 @@ def test_capacity_and_workspace(L):
     assert ws > 0 and ws % 16 == 0
 
 
+@pytest.mark.parametrize("key", sorted(W.WORKLOADS))
+def test_workspace_size_covers_every_sample_count(L, key):
+    """svg_workspace_size is the scratch of the workspace-taking calls for any
+    n in 1..64, and 0 on invalid arguments."""
+    pb = api.Problem.from_workload(W.WORKLOADS[key])
+    ws = api.workspace_size(pb)
+    assert ws > 0
+    assert all(api.profile_workspace_size(pb, n) <= ws for n in (1, 7, 32, 64))
+    sh, pr = pb.c_shape(), pb.c_params()
+    assert L.svg_workspace_size(None, ctypes.byref(pr)) == 0
+    assert L.svg_workspace_size(ctypes.byref(sh), None) == 0
+    pr.block_k = 32
+    assert L.svg_workspace_size(ctypes.byref(sh), ctypes.byref(pr)) == 0
+
+
+def test_release_with_nothing_cached_touches_no_gpu(L):
+    """With no host-buffer step run in this process nothing is cached, so the
+    call returns SVG_OK without any CUDA call (this machine may have no GPU)."""
+    assert L.svg_release() == 0
+    assert L.svg_release() == 0
+
+
 def _call_attn(L, sh, pr, ptr=16):
     p = ctypes.c_void_p(ptr)
     return L.svg_block_sparse_attn(ctypes.byref(sh), ctypes.byref(pr), p, p, p, p, p, p, p,

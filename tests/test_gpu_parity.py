@@ -386,6 +386,24 @@ def test_host_step_groups_match_one_shot_step(key, groups):
     assert torch.equal(kinds_h, buf.kinds.cpu())
 
 
+def test_release_then_host_step_again():
+    """svg_release frees the host step's streams, events and pinned staging;
+    the next host step creates them again and gives the same bits."""
+    wl, inp, _, _ = case("wan")
+    pb = pb_of(wl)
+    pin = lambda a: torch.from_numpy(a).view(torch.bfloat16).pin_memory()
+    args = (pin(inp["q"]), pin(inp["k"]), pin(inp["v"]), torch.from_numpy(inp["gamma_q"]).pin_memory(),
+            torch.from_numpy(inp["gamma_k"]).pin_memory(), torch.from_numpy(inp["sample_idx"]).pin_memory())
+    first = svg.HostStep(pb, wl.n_samples, groups=3)(*args)
+    torch.cuda.synchronize()
+    first = first.clone()
+    svg.release()
+    second = svg.HostStep(pb, wl.n_samples, groups=3)(*args)
+    torch.cuda.synchronize()
+    assert torch.equal(first.view(torch.int16), second.view(torch.int16))
+    svg.release()
+
+
 def test_host_buffer_api_matches_device_api():
     wl, inp, _, _ = case("tiny")
     pb = pb_of(wl)
