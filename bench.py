@@ -83,6 +83,22 @@ def reduce_over_ranks(times, work, device="cpu"):
     return [float(x) for x in t.cpu()], [float(x) for x in w.cpu()]
 
 
+def executed_tile_flops(row_ptr: np.ndarray, col: np.ndarray, wl) -> float:
+    """FLOPs the attention kernel's tensor cores execute for this block list.
+    With 128-row query tiles a CTA walks the union of its two tiles' lists and
+    runs S and P.V for both tiles on every block in it (a block listed for one
+    tile only is masked for the other), over whole 128x64 tiles; with 64-row
+    tiles each listed tile is computed whole."""
+    counts = np.diff(row_ptr.astype(np.int64))
+    if wl.bq != 128:
+        return float(4.0 * wl.d * wl.bq * wl.bk * counts.sum())
+    nqb, nkb = wl.nqb, wl.nkb
+    t = np.repeat(np.arange(counts.size, dtype=np.int64), counts)      # q-tile of each entry
+    pair = (t // nqb) * ((nqb + 1) // 2) + (t % nqb) // 2
+    union = np.unique(pair * (nkb + 1) + col.astype(np.int64)).size
+    return float(union * 2 * 4.0 * wl.d * wl.bq * wl.bk)
+
+
 def kept_tile_flops(row_ptr: np.ndarray, col: np.ndarray, wl) -> float:
     """4*d*rows*cols summed over the listed (q-block, k-block) tiles."""
     nqb = wl.nqb
@@ -248,6 +264,7 @@ def run_gpu(args, rank, world, local_rank):
         one_step()
     svg.sync_status()
     flops = kept_tile_flops(buf.row_ptr.cpu().numpy(), buf.col[: int(buf.row_ptr[-1])].cpu().numpy(), wl)
+    exec_flops = executed_tile_flops(buf.row_ptr.cpu().numpy(), buf.col[: int(buf.row_ptr[-1])].cpu().numpy(), wl)
     kinds = buf.kinds.cpu().numpy()
 
     if world > 1:
@@ -348,6 +365,8 @@ def run_gpu(args, rank, world, local_rank):
             "tile": f"{wl.bq}x{wl.bk}", "profiled_rows": wl.n_samples,
             "head_kinds": {"spatial": int((kinds == 0).sum()), "temporal": int((kinds == 1).sum())},
             "kept_tile_tflop": round(flops / 1e12, 4),
+            "executed_tile_tflop": round(exec_flops / 1e12, 4),
+            "union_walk_overhead": round(exec_flops / flops - 1.0, 4) if flops > 0 else None,
             "l2": "no flush: each step reads > 2 GB of inputs, far above the 126 MB L2",
             "parallelism": f"replicas x{world} (one independent layer per GPU)",
         },
