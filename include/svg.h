@@ -432,14 +432,16 @@ int64_t svg_block_index_capacity(const svg_shape* shape, const svg_params* param
 /* Device scratch bytes svg_profile_heads needs for n sampled rows. */
 size_t svg_profile_workspace_size(const svg_shape* shape, int n);
 
-/* Device scratch bytes that every entry point taking a caller workspace needs
+/* (Not on the pages: a sizing helper of this library's boundary.)
+ * Device scratch bytes that every entry point taking a caller workspace needs
  * for this shape and parameters: svg_profile_heads and svg_profile_heads_raw_q
  * with any n from 1 to 64 (the scratch does not grow with n).  0 for a null
  * pointer, a shape the library rejects, negative window parameters, or tiles
  * other than block_k = 64 and block_q in {64, 128}. */
 size_t svg_workspace_size(const svg_shape* shape, const svg_params* params);
 
-/* Releases the library's cached state: on every device that has run
+/* (Not on the pages: resource management of this library.)
+ * Releases the library's cached state: on every device that has run
  * svg_attention_step_host, it waits for the library's own three streams to
  * finish, then destroys them and their events and frees the pinned staging
  * buffer of the RoPE table.  Nothing else is cached (the fixed scratch of
